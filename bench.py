@@ -1,0 +1,428 @@
+"""Benchmark of the Sol-Attn forward (pool + fused forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload wan_75k] [--beta B]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+solattn_pool (block means, key covariance, mu/sigma) followed by
+solattn_forward (on-the-fly routing, exact kept blocks, zeroth-order correction)
+at the Wan2.1-14B-like 720p shape: 75,600 tokens (21x45x80 latent grid), 40
+heads, d = 128, beta calibrated for a 15 % mean kept-block density.
+
+Prints one JSON line. value = kept-block TFLOP/s of the whole step (kept-block
+FLOPs = 4 d n_i n_j summed over kept (i, j) pairs), whole job over all ranks.
+Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
+GPU (heads are independent; no collective on the data path); timing is the max
+over ranks.
+
+--impl reference runs the CPU oracle (the only other implementation of this
+method available here) on the host cores, on a bounded sample of the same
+workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_cov_b200.inputs import WORKLOADS, make_qkv  # noqa: E402
+
+METRIC = "Sol-Attn fwd ms & kept-block TFLOP/s (% BF16 peak) at 75.6K tokens, 1×B200"
+UNIT = "TFLOP/s (kept-block)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS)
+
+
+def load_beta(workload, target=None):
+    p = os.path.join(ROOT, "tests", "golden", "calibrated_beta.json")
+    d = json.load(open(p))[workload]
+    if target is None:
+        return d["beta"], d
+    return d["targets"][f"{target:.2f}"]["beta"], d
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- helpers
+def kept_flops(stats, dens, beta, N, d):
+    """Algorithmic kept-block FLOPs: 4 d n_i sum_{j in S_i} n_j over every (b, h, i).
+    Only the last key block can be partial; whether it is kept by row i is
+    recomputed from the pooled statistics (bookkeeping only)."""
+    nb = math.ceil(N / 64)
+    n_last = N - 64 * (nb - 1)
+    n_i = torch.full((nb,), 64.0, device=dens.device, dtype=torch.float64)
+    n_i[-1] = n_last
+    cols = 64.0 * dens.double()
+    if n_last < 64:
+        qbar, kbar = stats.view("qbar"), stats.view("kbar")
+        sh = (qbar.double() @ kbar[..., -1, :].double().unsqueeze(-1)).squeeze(-1) / math.sqrt(d)
+        tau = stats.view("mu").double() + beta * stats.view("sigma").double()
+        cols = cols - (64 - n_last) * (sh > tau).double()
+    return float((4.0 * d * n_i * cols).sum().item())
+
+
+def dense_flops(B, H, N, d):
+    return 4.0 * d * N * N * B * H
+
+
+def pool_bytes(B, H, N, d):
+    nb = math.ceil(N / 64)
+    return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d + 2 * nb) * B * H * 4
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [x.get("num_threads", 1) for x in threadpool_info() if x.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_sample(q, k, v, beta, heads, blocks_per_head, seed=0):
+    """Times the oracle on a stratified sample: per head, the first and last
+    query block plus random ones. Returns (seconds, kept FLOPs of the sample,
+    description)."""
+    from oracle import solattn_oracle as orc
+
+    N, d = q.shape[2], q.shape[3]
+    nb = math.ceil(N / 64)
+    rng = np.random.default_rng(seed)
+    t_total, flops = 0.0, 0.0
+    for h in heads:
+        rows = sorted({0, nb - 1, *rng.choice(nb, max(0, blocks_per_head - 2), replace=False).tolist()})
+        qq, kk, vv = (x[0, h].double().numpy() for x in (q, k, v))
+        t0 = time.perf_counter()
+        _, _, dens = orc.attend(qq, kk, vv, beta, rows=rows)
+        t_total += time.perf_counter() - t0
+        r = orc.route(qq, kk, beta)
+        n = orc.block_counts(N).astype(np.float64)
+        for i in rows:
+            flops += 4.0 * d * n[i] * float(n[r["mask"][i]].sum())
+    desc = f"oracle fp64 on {len(heads)} head(s) x {blocks_per_head} query blocks (first, last, random)"
+    return t_total, flops, desc
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    beta = args.beta if args.beta is not None else load_beta(args.workload)[0]
+    q, k, v = make_qkv(wl, 0, heads=[(0, 0)])
+    times, flops = [], 0.0
+    for step in range(args.warmup + args.steps):
+        t, f, desc = oracle_sample(q, k, v, beta, [0], 4, seed=step)
+        if step >= args.warmup:
+            times.append(t)
+            flops += f
+    secs = sum(times)
+    val = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "beta": beta,
+                   "sample": desc},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import block_sparse_attention_cov_b200 as sa
+    from block_sparse_attention_cov_b200 import _lib
+
+    _lib.lib()  # fail loudly if the extension is missing
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    beta = args.beta if args.beta is not None else load_beta(args.workload)[0]
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    peaks = load_peaks()
+
+    q_h, k_h, v_h = make_qkv(wl, seed=0)
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    stream = torch.cuda.current_stream()
+    ws = sa.workspace(dev)
+    stats = sa.pool(q, k, v)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    nb = math.ceil(N / 64)
+    dens = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sa.pool(q, k, v, stats)
+        if ev is not None:
+            ev[1].record(stream)
+        sa.forward(q, k, v, stats, beta, out=out, lse=lse, density=dens, ws=ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sa.status(ws) != 0:
+        raise RuntimeError(f"device status {sa.status(ws)} after warm-up")
+    kflops = kept_flops(stats, dens, beta, N, d)
+    mean_density = float(dens.double().mean().item()) / nb
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank] if cvd else str(local_rank))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    st = sa.status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the timed region")
+    ms_total = t_start.elapsed_time(t_end)
+    pool_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    fwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = torch.tensor([ms_total, pool_ms, fwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
+    ms_total, pool_ms, fwd_ms = (float(x) for x in ms.tolist())
+    ms_step = ms_total / args.steps
+
+    # dense comparison path on the same inputs
+    dense_ms = None
+    if not args.skip_dense:
+        sa.dense(q, k, v, out=out, lse=lse, ws=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        reps = 2
+        for _ in range(reps):
+            sa.dense(q, k, v, out=out, lse=lse, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / reps
+        step()  # restore the Sol-Attn outputs
+        torch.cuda.synchronize()
+
+    # end to end: pinned host inputs -> device -> pool + forward -> host outputs
+    e2e = None
+    if not args.skip_e2e:
+        qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dens_h = torch.empty(dens.shape, dtype=dens.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qp, non_blocking=True)
+            kd.copy_(kp, non_blocking=True)
+            vd.copy_(vp, non_blocking=True)
+            sa.pool(qd, kd, vd, stats)
+            sa.forward(qd, kd, vd, stats, beta, out=out, lse=lse, density=dens, ws=ws)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+            dens_h.copy_(dens, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        reps = max(1, min(args.steps, 3))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([e0.elapsed_time(e1) / reps], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp))
+        d2h = sum(x.numel() * x.element_size() for x in (out_h, lse_h, dens_h))
+        e2e = {"value": world * kflops / (float(e2e_ms.item()) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(e2e_ms.item())}
+
+    if rank != 0:
+        return
+
+    fwd_tflops = kflops / (fwd_ms * 1e-3) / 1e12
+    pbytes = pool_bytes(B, H, N, d)
+    pool_gbs = pbytes / (pool_ms * 1e-3) / 1e9
+    cpu = None
+    if not args.skip_cpu and world == 1:
+        secs, fl, desc = oracle_sample(q_h, k_h, v_h, beta, [0, H // 2], args.cpu_blocks)
+        cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": desc + f"; {secs:.1f} s of CPU time"}
+    line = {
+        "metric": METRIC,
+        "value": world * kflops / (ms_step * 1e-3) / 1e12,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; bf16)",
+        "config": {
+            "workload": args.workload, "B": B, "H": H, "N": N, "d": d, "grid": list(wl.grid), "beta": beta,
+            "mean_density": mean_density, "global_batch": B * world, "seq_len": N,
+            "parallelism": f"heads-independent replicas x{world}",
+            "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no explicit flush" % (B * H * N * d * 2 / 1e6),
+        },
+        "fwd_ms": fwd_ms,
+        "pool_ms": pool_ms,
+        "fwd_kept_tflops": fwd_tflops,
+        "fwd_frac_bf16_peak": fwd_tflops / peaks["bf16_tflops"],
+        "fwd_frac_bf16_sustained": fwd_tflops / peaks["bf16_tflops_sustained"],
+        "pool_gbs": pool_gbs,
+        "pool_frac_hbm": pool_gbs / peaks["hbm_gbs"],
+        "dense_ms": dense_ms,
+        "speedup_vs_dense": (dense_ms / fwd_ms) if dense_ms else None,
+        "kept_tflop_per_step": kflops / 1e12,
+        "roofline": {
+            "bound": "tensor",
+            "achieved": fwd_tflops,
+            "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": fwd_tflops / peaks["bf16_tflops"],
+            "traffic": None,
+            "kernel": "solattn_fwd_kernel (fused forward)",
+            "peak_source": peaks["source"] + " (bf16 burst)",
+        },
+        "pool_roofline": {
+            "bound": "hbm", "achieved": pool_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": pool_gbs / peaks["hbm_gbs"], "algorithmic_bytes": pbytes,
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk,
+        "gpu_launches": 4 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan_75k", choices=sorted(WORKLOADS))
+    ap.add_argument("--beta", type=float, default=None)
+    ap.add_argument("--cpu-blocks", type=int, default=24)
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-dense", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

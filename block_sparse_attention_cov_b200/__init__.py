@@ -1,0 +1,145 @@
+"""Sol-Attn block-sparse attention forward for B200 (sm_100a).
+
+Python binding of the C ABI in include/solattn.h: argument marshalling only
+(torch tensors -> device pointers, the current CUDA stream, output allocation).
+Every step of the computation runs in the library's CUDA kernels; there is no
+CPU path. The names mirror the C calls:
+
+    stats = pool(q, k, v)                          # solattn_pool
+    out, lse, density = forward(q, k, v, stats, beta)   # solattn_forward
+    out, lse = dense(q, k, v)                      # solattn_dense
+
+q, k, v: CUDA bf16 tensors [B, H, N, d], contiguous, d in {64, 128}.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+__all__ = ["SolAttnError", "PooledStats", "pool", "forward", "dense", "status", "workspace", "pooled_bytes"]
+
+
+class SolAttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = int(code)
+        super().__init__(f"{what}: {_lib.strerror(code)} (code {code})")
+
+
+def _check(rc: int, what: str):
+    if rc != _lib.OK:
+        raise SolAttnError(rc, what)
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous CUDA bf16 tensors [B, H, N, d]")
+    if not all(t.shape == ts[0].shape for t in ts):
+        raise ValueError("q, k, v must have the same shape")
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def pooled_bytes(B: int, H: int, N: int, d: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.lib().solattn_pooled_layout(B, H, N, d, None, None, ctypes.byref(n)), "solattn_pooled_layout")
+    return int(n.value)
+
+
+@dataclass
+class PooledStats:
+    """solattn_pool's outputs: one device buffer and fp32 views into it."""
+
+    buffer: torch.Tensor
+    struct: _lib.PooledStruct
+    shape: tuple
+
+    def view(self, name: str) -> torch.Tensor:
+        B, H, N, d = self.shape
+        nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
+        dims = {
+            "qbar": (B, H, nb, d), "kbar": (B, H, nb, d), "vbar": (B, H, nb, d),
+            "kmean": (B, H, d), "kcov": (B, H, d, d), "mu": (B, H, nb), "sigma": (B, H, nb),
+        }[name]
+        off = getattr(self.struct, name) - self.buffer.data_ptr()
+        n = math.prod(dims)
+        return self.buffer[off:off + 4 * n].view(torch.float32).view(dims)
+
+
+def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stats: PooledStats | None = None) -> PooledStats:
+    """Block means of q, k, v and the key mean/covariance, mu and sigma (solattn_pool)."""
+    _check_inputs(q, k, v)
+    B, H, N, d = _shape(q)
+    if stats is None:
+        nbytes = pooled_bytes(B, H, N, d)
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+        st = _lib.PooledStruct()
+        _check(_lib.lib().solattn_pooled_layout(B, H, N, d, _ptr(buf), ctypes.byref(st), None),
+               "solattn_pooled_layout")
+        stats = PooledStats(buf, st, (B, H, N, d))
+    elif stats.shape != (B, H, N, d):
+        raise ValueError("PooledStats shape does not match the inputs")
+    _check(_lib.lib().solattn_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct), _stream()),
+           "solattn_pool")
+    return stats
+
+
+def workspace(device=None) -> torch.Tensor:
+    """A device workspace for forward/dense (scheduler counter and status word)."""
+    return torch.empty(_lib.WORKSPACE_BYTES, dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(q, k, v, stats: PooledStats, beta: float, out=None, lse=None, density=None, ws=None,
+            want_lse: bool = True, want_density: bool = True):
+    """Sol-Attn forward (solattn_forward). Returns (out, lse, density)."""
+    _check_inputs(q, k, v)
+    B, H, N, d = _shape(q)
+    nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if density is None and want_density:
+        density = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
+    ws = workspace(q.device) if ws is None else ws
+    rc = _lib.lib().solattn_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
+                                    ctypes.c_float(beta), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
+                                    ws.numel(), _stream())
+    _check(rc, "solattn_forward")
+    return out, lse, density
+
+
+def dense(q, k, v, out=None, lse=None, ws=None, want_lse: bool = True):
+    """Dense attention through the same kernel with routing off (solattn_dense)."""
+    _check_inputs(q, k, v)
+    B, H, N, d = _shape(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ws = workspace(q.device) if ws is None else ws
+    rc = _lib.lib().solattn_dense(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(out), _ptr(lse), _ptr(ws),
+                                  ws.numel(), _stream())
+    _check(rc, "solattn_dense")
+    return out, lse
+
+
+def status(ws: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the device status of the last
+    call that used `ws` (0 = ok, 5 = a bounded wait expired)."""
+    return int(_lib.lib().solattn_status(_ptr(ws), _stream()))

@@ -1,0 +1,72 @@
+"""ctypes loader for libsolattn.so (the C ABI of include/solattn.h)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+
+# Every symbol declared in include/solattn.h.
+EXPORTS = (
+    "solattn_pooled_layout",
+    "solattn_pool",
+    "solattn_forward",
+    "solattn_dense",
+    "solattn_status",
+    "solattn_strerror",
+    "solattn_version",
+)
+
+OK = 0
+ERR_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_ALIGN = 3
+ERR_CUDA = 4
+ERR_TIMEOUT = 5
+ERR_DEVICE = 6
+ERR_WORKSPACE = 7
+WORKSPACE_BYTES = 256
+BLOCK = 64
+MAX_TOKENS = 262144
+
+
+class PooledStruct(ctypes.Structure):
+    """Mirror of solattn_pooled_t."""
+
+    _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov", "mu", "sigma")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library. Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing; build it with `python -m block_sparse_attention_cov_b200.build`"
+        )
+    L = ctypes.CDLL(LIB_PATH)
+    i, vp, f, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+    L.solattn_pooled_layout.argtypes = [i, i, i, i, vp, ctypes.POINTER(PooledStruct), ctypes.POINTER(sz)]
+    L.solattn_pooled_layout.restype = i
+    L.solattn_pool.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(PooledStruct), vp]
+    L.solattn_pool.restype = i
+    L.solattn_forward.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(PooledStruct), f, vp, vp, vp, vp, sz, vp]
+    L.solattn_forward.restype = i
+    L.solattn_dense.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, sz, vp]
+    L.solattn_dense.restype = i
+    L.solattn_status.argtypes = [vp, vp]
+    L.solattn_status.restype = i
+    L.solattn_strerror.argtypes = [i]
+    L.solattn_strerror.restype = ctypes.c_char_p
+    L.solattn_version.argtypes = []
+    L.solattn_version.restype = i
+    _lib = L
+    return L
+
+
+def strerror(code: int) -> str:
+    return lib().solattn_strerror(int(code)).decode()

@@ -1,0 +1,200 @@
+// api.cu -- the C ABI declared in include/solattn.h: argument checks, buffer
+// layout helpers and stream-ordered launches. No allocation happens here.
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/solattn.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace {
+
+using solattn::DeviceStatus;
+using solattn::PooledPtrs;
+
+static_assert(sizeof(DeviceStatus) <= SOLATTN_WORKSPACE_BYTES, "workspace too small for the status block");
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];   // 0 = not yet queried, -1 = not an sm_100 device
+int g_cc[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_shape(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SOLATTN_ERR_ARG;
+  if (d != 64 && d != 128) return SOLATTN_ERR_UNSUPPORTED;
+  if (N > SOLATTN_MAX_TOKENS) return SOLATTN_ERR_UNSUPPORTED;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long nb = (N + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
+  if (bh * ((nb + 1) / 2) >= (1ll << 31) || bh >= (1ll << 31)) return SOLATTN_ERR_UNSUPPORTED;
+  return SOLATTN_OK;
+}
+
+int check_qkv(const void* q, const void* k, const void* v) {
+  if (!q || !k || !v) return SOLATTN_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SOLATTN_ERR_ALIGN;
+  return SOLATTN_OK;
+}
+
+int check_pooled(const solattn_pooled_t* p) {
+  if (!p) return SOLATTN_ERR_ARG;
+  const void* ptrs[7] = {p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, p->mu, p->sigma};
+  for (const void* x : ptrs)
+    if (!x) return SOLATTN_ERR_ARG;
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return SOLATTN_ERR_ALIGN;
+  return SOLATTN_OK;
+}
+
+// Multiprocessor count of the current device, or an error code (negative).
+int current_device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SOLATTN_ERR_DEVICE;
+  if (g_sms[dev] == 0) {
+    int major = 0, minor = 0, count = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SOLATTN_ERR_CUDA;
+    g_cc[dev] = major * 10 + minor;
+    g_sms[dev] = (major == 10 && minor == 0) ? count : -1;
+  }
+  if (g_sms[dev] < 0) return SOLATTN_ERR_DEVICE;
+  *sms = g_sms[dev];
+  return SOLATTN_OK;
+}
+
+PooledPtrs to_ptrs(const solattn_pooled_t* p) {
+  return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, p->mu, p->sigma};
+}
+
+int run_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                const solattn_pooled_t* pooled, float beta, bool route, void* out, float* lse, int32_t* density,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_qkv(q, k, v))) return rc;
+  if (!out) return SOLATTN_ERR_ARG;
+  if (!aligned16(out)) return SOLATTN_ERR_ALIGN;
+  if ((lse && !aligned4(lse)) || (density && !aligned4(density))) return SOLATTN_ERR_ALIGN;
+  if (route) {
+    if (std::isnan(beta)) return SOLATTN_ERR_ARG;
+    if ((rc = check_pooled(pooled))) return rc;
+  }
+  if (!workspace || workspace_bytes < SOLATTN_WORKSPACE_BYTES) return SOLATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SOLATTN_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = current_device_sms(&sms))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // scheduler counter and status word start at zero for every call
+  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), s) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  solattn::ForwardArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.density = route ? density : nullptr;
+  if (route) a.pooled = to_ptrs(pooled);
+  a.beta = beta;
+  a.route = route;
+  a.BH = B * H;
+  a.N = N;
+  a.d = d;
+  a.status = workspace;
+  return solattn::launch_forward(a, sms, s) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+int solattn_version(void) { return 10000; }
+
+const char* solattn_strerror(int code) {
+  switch (code) {
+    case SOLATTN_OK: return "ok";
+    case SOLATTN_ERR_ARG: return "invalid argument (null pointer, non-positive size or NaN beta)";
+    case SOLATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128, N <= 262144)";
+    case SOLATTN_ERR_ALIGN: return "device pointer not aligned (16 bytes for tensors, 4 for lse/density)";
+    case SOLATTN_ERR_CUDA: return "CUDA runtime error";
+    case SOLATTN_ERR_TIMEOUT: return "a bounded wait inside the kernel expired; outputs are invalid";
+    case SOLATTN_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    case SOLATTN_ERR_WORKSPACE: return "workspace missing or smaller than SOLATTN_WORKSPACE_BYTES";
+    default: return "unknown status code";
+  }
+}
+
+int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled_t* pooled, size_t* bytes) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (!bytes && !pooled) return SOLATTN_ERR_ARG;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t nb = (static_cast<size_t>(N) + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
+  const size_t f = sizeof(float);
+  const size_t sizes[7] = {bh * nb * d * f, bh * nb * d * f, bh * nb * d * f, bh * d * f,
+                           bh * static_cast<size_t>(d) * d * f, bh * nb * f, bh * nb * f};
+  size_t off[7], total = 0;
+  for (int i = 0; i < 7; ++i) {
+    off[i] = total;
+    total += round256(sizes[i]);
+  }
+  if (bytes) *bytes = total;
+  if (pooled && base) {
+    char* b = static_cast<char*>(base);
+    if (!aligned16(base)) return SOLATTN_ERR_ALIGN;
+    pooled->qbar = reinterpret_cast<float*>(b + off[0]);
+    pooled->kbar = reinterpret_cast<float*>(b + off[1]);
+    pooled->vbar = reinterpret_cast<float*>(b + off[2]);
+    pooled->kmean = reinterpret_cast<float*>(b + off[3]);
+    pooled->kcov = reinterpret_cast<float*>(b + off[4]);
+    pooled->mu = reinterpret_cast<float*>(b + off[5]);
+    pooled->sigma = reinterpret_cast<float*>(b + off[6]);
+  } else if (pooled && !base) {
+    return SOLATTN_ERR_ARG;
+  }
+  return SOLATTN_OK;
+}
+
+int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                 const solattn_pooled_t* pooled, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_qkv(q, k, v))) return rc;
+  if ((rc = check_pooled(pooled))) return rc;
+  int sms = 0;
+  if ((rc = current_device_sms(&sms))) return rc;
+  const cudaError_t e =
+      solattn::launch_pool(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                           static_cast<const uint16_t*>(v), to_ptrs(pooled), B * H, N, d, sms,
+                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+}
+
+int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                    const solattn_pooled_t* pooled, float beta, void* out, float* lse, int32_t* density_out,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return run_forward(q, k, v, B, H, N, d, pooled, beta, true, out, lse, density_out, workspace, workspace_bytes,
+                     stream);
+}
+
+int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int N, int d, void* out, float* lse,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  return run_forward(q, k, v, B, H, N, d, nullptr, -INFINITY, false, out, lse, nullptr, workspace,
+                     workspace_bytes, stream);
+}
+
+int solattn_status(const void* workspace, void* stream) {
+  if (!workspace) return SOLATTN_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  DeviceStatus h{};
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  return h.error == 0 ? SOLATTN_OK : static_cast<int>(h.error);
+}
+
+}  // extern "C"

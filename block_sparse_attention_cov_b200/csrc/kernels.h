@@ -1,0 +1,39 @@
+// kernels.h -- internal launch interface between the C ABI layer and the CUDA
+// kernels (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace solattn {
+
+struct PooledPtrs {
+  float* qbar;
+  float* kbar;
+  float* vbar;
+  float* kmean;
+  float* kcov;
+  float* mu;
+  float* sigma;
+};
+
+struct ForwardArgs {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  uint16_t* out;
+  float* lse;          // may be null
+  int32_t* density;    // may be null
+  PooledPtrs pooled;   // unused when route == false
+  float beta;
+  bool route;          // false: dense attention (no routing, no correction)
+  int BH, N, d;
+  void* status;        // DeviceStatus in the caller's workspace
+};
+
+cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, const PooledPtrs& p, int BH,
+                        int N, int d, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace solattn

@@ -1,0 +1,157 @@
+/*
+ * solattn.h -- C ABI of the Sol-Attn block-sparse attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is Sol-Attn ("Sol-Attn: Accelerating Video Generation Inference
+ * via On-the-Fly Attention Sparsification", arXiv 2607.24027), as described on
+ * the pages hotpaper.ai (abstract), agihunt.info (digest) and paithon.it
+ * (article). Section names below are the paithon.it headings.
+ *
+ * Notation: B batch, H heads, N tokens, d head dimension (64 or 128),
+ * 64-token blocks ("Perché l'attenzione pesa tanto nei video"),
+ * N_b = ceil(N / 64), n_j = valid tokens of block j (64, or fewer for the last),
+ * s = 1/sqrt(d).
+ *
+ * Layouts (row-major, contiguous, no padding):
+ *   q, k, v, out        bf16 [B][H][N][d]   (passed as raw 16-bit words)
+ *   lse                 fp32 [B][H][N]      natural log of the softmax sum
+ *   density_out         int32 [B][H][N_b]   |S_i| = kept key blocks per query block
+ *   pooled buffers      fp32, see solattn_pooled_t
+ *
+ * Ownership: the caller allocates every buffer, on the device unless a function
+ * says otherwise. No call allocates device memory. Nothing is retained after a
+ * call returns. Every device pointer must be 16-byte aligned.
+ *
+ * Ordering: every call that takes `stream` (a cudaStream_t, NULL = legacy
+ * default stream) is asynchronous on that stream and returns once its work is
+ * enqueued. Argument errors are reported before anything is enqueued.
+ *
+ * Errors: every int-returning call returns SOLATTN_OK (0) or one of the codes
+ * below; solattn_strerror() names them. Errors that happen on the device (a
+ * bounded wait that expired) are recorded in the caller's workspace and
+ * reported by solattn_status().
+ */
+#ifndef SOLATTN_H_
+#define SOLATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SOLATTN_BLOCK 64          /* tokens per block */
+#define SOLATTN_MAX_TOKENS 262144 /* N limit (N_b <= 4096) */
+#define SOLATTN_WORKSPACE_BYTES 256
+
+enum solattn_status_code {
+  SOLATTN_OK = 0,
+  SOLATTN_ERR_ARG = 1,         /* null pointer, non-positive size, NaN beta */
+  SOLATTN_ERR_UNSUPPORTED = 2, /* d not in {64,128}, N > SOLATTN_MAX_TOKENS, B*H too large */
+  SOLATTN_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+  SOLATTN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  SOLATTN_ERR_TIMEOUT = 5,     /* a bounded device wait expired (device side) */
+  SOLATTN_ERR_DEVICE = 6,      /* current device is not an sm_100 GPU */
+  SOLATTN_ERR_WORKSPACE = 7    /* workspace missing or smaller than SOLATTN_WORKSPACE_BYTES */
+};
+
+/*
+ * Pooled statistics of one (q, k, v) triple, written by solattn_pool and read
+ * by solattn_forward. All fp32, device memory, caller-owned:
+ *   qbar, kbar, vbar  [B][H][N_b][d]  block means over valid tokens
+ *   kmean             [B][H][d]       mean of the pooled keys (each block counts once)
+ *   kcov              [B][H][d][d]    covariance of the pooled keys, divided by N_b
+ *   mu, sigma         [B][H][N_b]     mean and population standard deviation of
+ *                                     every proxy row s_hat_i. (paithon.it,
+ *                                     "Una soglia per ogni riga": the threshold's
+ *                                     statistics come from the key mean and the
+ *                                     d x d second-moment matrix.)
+ */
+typedef struct {
+  float* qbar;
+  float* kbar;
+  float* vbar;
+  float* kmean;
+  float* kcov;
+  float* mu;
+  float* sigma;
+} solattn_pooled_t;
+
+/*
+ * Size in bytes of one contiguous buffer holding every pooled array, and (when
+ * base != NULL) the pointers into it, each 256-byte aligned. base may be a
+ * device pointer; it is only used for address arithmetic, never dereferenced.
+ * Host-only; enqueues nothing.
+ */
+int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled_t* pooled,
+                          size_t* bytes);
+
+/*
+ * Pooling (paithon.it, "Perché l'attenzione pesa tanto nei video": proxy scores
+ * are products of block-mean queries and keys; "Una soglia per ogni riga",
+ * last paragraph: mu_i and sigma_i from the mean and d x d second-moment matrix
+ * of the pooled keys).
+ * Reads q, k, v once and writes every array of `pooled` (the struct itself is
+ * host memory, its pointers are device memory):
+ *   qbar_i = mean of the valid query tokens of block i (likewise kbar, vbar);
+ *   kmean  = (1/N_b) sum_j kbar_j;
+ *   kcov   = (1/N_b) sum_j (kbar_j - kmean)(kbar_j - kmean)^T;
+ *   mu_i   = s qbar_i . kmean;   sigma_i = s sqrt(max(0, qbar_i^T kcov qbar_i)).
+ */
+int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                 const solattn_pooled_t* pooled, void* stream);
+
+/*
+ * Sol-Attn forward (hotpaper.ai abstract: routing, sparse computation and
+ * correction in one online-softmax pass; paithon.it "Una soglia per ogni riga":
+ * tau_i = mu_i + beta sigma_i, S_i = {j : s_hat_ij > tau_i}; "Scegliere mentre si
+ * calcola": proxy scores compared with tau_i as they are produced, kept blocks
+ * attended exactly, skipped blocks approximated by the zeroth-order Taylor term
+ * that reuses their proxy scores, both in the same softmax state).
+ *
+ * For every query token t of block i, with s_hat_ij = s qbar_i . kbar_j:
+ *   out_t = (sum_{j in S_i} sum_{u in j} e^{s q_t.k_u} v_u + sum_{j not in S_i} n_j e^{s_hat_ij} vbar_j)
+ *         / (sum_{j in S_i} sum_{u in j} e^{s q_t.k_u}     + sum_{j not in S_i} n_j e^{s_hat_ij})
+ *   lse_t = natural log of the denominator;   density_out_i = |S_i|.
+ * beta = -INFINITY keeps every block (dense attention); beta = +INFINITY skips
+ * every block. The proxy map s_hat is never written to memory.
+ *
+ * pooled must hold solattn_pool's results for the same q and k. lse and
+ * density_out may be NULL. workspace: device memory of at least
+ * SOLATTN_WORKSPACE_BYTES, owned by the caller, used by one call at a time
+ * (calls sharing a workspace must not overlap on the device); its contents
+ * need no initialisation and are rewritten by every call.
+ */
+int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                    const solattn_pooled_t* pooled, float beta, void* out, float* lse,
+                    int32_t* density_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dense softmax attention with scale 1/sqrt(d) by the same kernel with routing
+ * switched off: equal to solattn_forward with beta = -INFINITY, without the
+ * pooled statistics. lse may be NULL. workspace as for solattn_forward.
+ */
+int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int N, int d, void* out,
+                  float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns the device-side status recorded in
+ * `workspace` by the last forward or dense call that used it: SOLATTN_OK or
+ * SOLATTN_ERR_TIMEOUT (a bounded wait inside the kernel gave up; the kernel
+ * returned early and its outputs are invalid). SOLATTN_ERR_CUDA if the
+ * synchronisation or the read fails.
+ */
+int solattn_status(const void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* solattn_strerror(int code);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int solattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOLATTN_H_ */

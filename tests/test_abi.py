@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/solattn.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_cov_b200 import _lib
+from block_sparse_attention_cov_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "solattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(solattn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_python_export_list():
+    assert _declared() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_version_and_strerror(L):
+    assert L.solattn_version() == 10000
+    for code in range(0, 8):
+        assert _lib.strerror(code) and "unknown" not in _lib.strerror(code)
+    assert "unknown" in _lib.strerror(99)
+
+
+def _pooled_struct(addr=0x100000):
+    st = _lib.PooledStruct()
+    for i, (name, _) in enumerate(_lib.PooledStruct._fields_):
+        setattr(st, name, addr + i * 0x10000)
+    return st
+
+
+FAKE = ctypes.c_void_p(0x7F0000000000)  # never dereferenced: every call below fails validation first
+
+
+def _fwd(L, q=FAKE, k=FAKE, v=FAKE, B=1, H=1, N=128, d=64, pooled=None, beta=0.5, out=FAKE, lse=None,
+         dens=None, ws=FAKE, wsb=256):
+    pooled = _pooled_struct() if pooled is None else pooled
+    return L.solattn_forward(q, k, v, B, H, N, d, ctypes.byref(pooled), ctypes.c_float(beta), out, lse, dens,
+                             ws, wsb, None)
+
+
+def test_forward_argument_errors(L):
+    assert _fwd(L, q=None) == _lib.ERR_ARG
+    assert _fwd(L, out=None) == _lib.ERR_ARG
+    assert _fwd(L, N=0) == _lib.ERR_ARG
+    assert _fwd(L, B=-1) == _lib.ERR_ARG
+    assert _fwd(L, d=96) == _lib.ERR_UNSUPPORTED
+    assert _fwd(L, N=_lib.MAX_TOKENS + 1) == _lib.ERR_UNSUPPORTED
+    assert _fwd(L, beta=math.nan) == _lib.ERR_ARG
+    assert _fwd(L, k=ctypes.c_void_p(0x7F0000000008)) == _lib.ERR_ALIGN
+    assert _fwd(L, lse=ctypes.c_void_p(0x7F0000000002)) == _lib.ERR_ALIGN
+    bad = _pooled_struct()
+    bad.mu = None
+    assert _fwd(L, pooled=bad) == _lib.ERR_ARG
+    bad = _pooled_struct()
+    bad.kcov = 0x100004
+    assert _fwd(L, pooled=bad) == _lib.ERR_ALIGN
+    assert _fwd(L, ws=None) == _lib.ERR_WORKSPACE
+    assert _fwd(L, wsb=255) == _lib.ERR_WORKSPACE
+
+
+def test_dense_and_pool_argument_errors(L):
+    assert L.solattn_dense(FAKE, FAKE, None, 1, 1, 64, 128, FAKE, None, FAKE, 256, None) == _lib.ERR_ARG
+    assert L.solattn_dense(FAKE, FAKE, FAKE, 1, 1, 64, 32, FAKE, None, FAKE, 256, None) == _lib.ERR_UNSUPPORTED
+    assert L.solattn_dense(FAKE, FAKE, FAKE, 1, 1, 64, 128, FAKE, None, None, 256, None) == _lib.ERR_WORKSPACE
+    st = _pooled_struct()
+    assert L.solattn_pool(FAKE, FAKE, FAKE, 1, 1, 0, 64, ctypes.byref(st), None) == _lib.ERR_ARG
+    assert L.solattn_pool(FAKE, FAKE, FAKE, 1, 1, 64, 64, None, None) == _lib.ERR_ARG
+    assert L.solattn_status(None, None) == _lib.ERR_WORKSPACE
+
+
+def test_pooled_layout_sizes_and_alignment(L):
+    n = ctypes.c_size_t(0)
+    B, H, N, d = 1, 40, 75600, 128
+    assert L.solattn_pooled_layout(B, H, N, d, None, None, ctypes.byref(n)) == 0
+    nb = math.ceil(N / 64)
+    r = lambda x: (x + 255) // 256 * 256
+    want = 3 * r(B * H * nb * d * 4) + r(B * H * d * 4) + r(B * H * d * d * 4) + 2 * r(B * H * nb * 4)
+    assert n.value == want
+    st = _lib.PooledStruct()
+    base = 0x10000000
+    assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base), ctypes.byref(st), None) == 0
+    ptrs = [getattr(st, f) for f, _ in _lib.PooledStruct._fields_]
+    assert ptrs[0] == base and all(p % 256 == 0 for p in ptrs) and ptrs == sorted(ptrs)
+    assert ptrs[-1] + r(B * H * nb * 4) == base + want
+    assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base + 8), ctypes.byref(st), None) == _lib.ERR_ALIGN
+    assert L.solattn_pooled_layout(B, H, N, 80, None, None, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED

@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded bf16 inputs.
+
+Acceptance (Sol-Attn forward spec for this library):
+  * kept-block decisions: per query block, |S_i| equals the oracle's exactly,
+    except that blocks whose fp64 proxy score lies within 1e-4 of tau_i
+    ("near ties") may flip; those are counted and bound the difference;
+  * out (bf16) vs the fp64 oracle over valid rows: relative L2 <= 1e-2 and
+    max abs <= 2e-2;
+  * lse: max abs <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_cov_b200 as sa
+from block_sparse_attention_cov_b200.build import build
+from block_sparse_attention_cov_b200.inputs import WORKLOADS, Workload, make_qkv
+from oracle import solattn_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+REL_L2, MAX_ABS, LSE_ABS, TIE = 1e-2, 2e-2, 1e-3, 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build()
+    major, minor = torch.cuda.get_device_capability()
+    assert (major, minor) == (10, 0), "these kernels are built for sm_100a"
+
+
+def _dev(*ts):
+    return [t.cuda().contiguous() for t in ts]
+
+
+def _near_ties(q, k, beta):
+    """Per (b, h, i): number of key blocks with |s_hat - tau| <= 1e-4 (fp64)."""
+    r = orc.route_all(q, k, beta)
+    return (np.abs(r["shat"] - r["tau"][..., None]) <= TIE).sum(-1), r
+
+
+def _check_density(dens_gpu, dens_orc, ties):
+    diff = np.abs(dens_gpu.astype(np.int64) - dens_orc)
+    assert (diff[ties == 0] == 0).all(), "density differs on a block without near ties"
+    assert (diff <= ties).all(), "density differs by more than the near-tie count"
+
+
+def _check_out(out_gpu, lse_gpu, out_o, lse_o, rows_mask=None):
+    og = out_gpu.float().cpu().numpy().astype(np.float64)
+    lg = lse_gpu.cpu().numpy().astype(np.float64)
+    if rows_mask is not None:
+        og, out_o, lg, lse_o = og[rows_mask], out_o[rows_mask], lg[rows_mask], lse_o[rows_mask]
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    err = og - out_o
+    rel = np.linalg.norm(err) / np.linalg.norm(out_o)
+    mx = np.abs(err).max()
+    assert rel <= REL_L2 and mx <= MAX_ABS, (rel, mx)
+    assert np.abs(lg - lse_o).max() <= LSE_ABS, np.abs(lg - lse_o).max()
+    return rel, mx
+
+
+def _wl(B, H, d, N):
+    return Workload(f"r{B}x{H}x{N}x{d}", B, H, d, (1, 1, N))
+
+
+# --------------------------------------------------------------------------- pooling
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], WORKLOADS["mid"], _wl(2, 3, 128, 1000), _wl(1, 2, 64, 37)],
+                         ids=lambda w: w.name)
+def test_pool_matches_oracle(wl):
+    q, k, v = make_qkv(wl, seed=1)
+    st = sa.pool(*_dev(q, k, v))
+    torch.cuda.synchronize()
+    B, H = wl.B, wl.H
+    for b in range(B):
+        for h in range(H):
+            qq, kk, vv = (x[b, h].double().numpy() for x in (q, k, v))
+            r = orc.route(qq, kk, 0.0)
+            np.testing.assert_allclose(st.view("qbar")[b, h].cpu().numpy(), r["qbar"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(st.view("kbar")[b, h].cpu().numpy(), r["kbar"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(st.view("vbar")[b, h].cpu().numpy(), orc.pool(vv), rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(st.view("kmean")[b, h].cpu().numpy(), r["kmean"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(st.view("kcov")[b, h].cpu().numpy(), r["kcov"], rtol=1e-4, atol=1e-6)
+            np.testing.assert_allclose(st.view("mu")[b, h].cpu().numpy(), r["mu"], rtol=1e-4, atol=1e-6)
+            np.testing.assert_allclose(st.view("sigma")[b, h].cpu().numpy(), r["sigma"], rtol=1e-4, atol=1e-6)
+
+
+# --------------------------------------------------------------------------- forward
+CASES = [
+    ("tiny", WORKLOADS["tiny"], [-math.inf, 0.5, 1.0], None),
+    ("mid", WORKLOADS["mid"], [0.0, 0.5, 1.0, 1.5], [0, 1, 2, 31, 64, 100, 126, 127]),
+    ("ragged_d128_b2h3", _wl(2, 3, 128, 1000), [-math.inf, 0.0, 0.7, math.inf], None),
+    ("ragged_d64", _wl(1, 2, 64, 64 * 5 + 20), [0.3, math.inf], None),
+    ("odd_blocks", _wl(1, 2, 128, 64 * 3), [0.0, -math.inf], None),
+    ("single_partial_block", _wl(1, 1, 64, 37), [-math.inf, 0.0, math.inf], None),
+]
+
+
+@pytest.mark.parametrize("name,wl,betas,rows", CASES, ids=[c[0] for c in CASES])
+def test_forward_matches_oracle(name, wl, betas, rows):
+    q, k, v = make_qkv(wl, seed=2)
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    ws = sa.workspace()
+    nb = math.ceil(wl.N / 64)
+    for beta in betas:
+        out, lse, dens = sa.forward(qd, kd, vd, st, beta, ws=ws)
+        assert sa.status(ws) == 0
+        ties, r = _near_ties(q, k, beta)
+        _check_density(dens.cpu().numpy(), r["density"], ties)
+        out_o, lse_o, _ = orc.forward(q, k, v, beta, rows=rows)
+        mask = None
+        if rows is not None:
+            mask = np.zeros((wl.B, wl.H, wl.N), bool)
+            for i in rows:
+                mask[:, :, i * 64:min(wl.N, i * 64 + 64)] = True
+        _check_out(out, lse, out_o, lse_o, mask)
+
+
+def test_beta_minus_inf_equals_dense_path_bitwise_and_dense_matches_oracle():
+    wl = _wl(1, 2, 128, 64 * 9 + 5)
+    q, k, v = make_qkv(wl, seed=3)
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    o1, l1, d1 = sa.forward(qd, kd, vd, st, -math.inf)
+    o2, l2 = sa.dense(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert (d1.cpu() == math.ceil(wl.N / 64)).all()
+    for h in range(wl.H):
+        od, ld = orc.dense_attention(*(x[0, h].double().numpy() for x in (q, k, v)))
+        _check_out(o2[0, h], l2[0, h], od, ld)
+
+
+def test_repeated_calls_are_deterministic():
+    wl = WORKLOADS["mid"]
+    q, k, v = make_qkv(wl, seed=4, heads=[(0, 0), (0, 5)])
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    a = sa.forward(qd, kd, vd, st, 0.8)
+    b = sa.forward(qd, kd, vd, st, 0.8)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_density_is_monotone_in_beta():
+    wl = WORKLOADS["mid"]
+    q, k, v = make_qkv(wl, seed=5, heads=[(0, 1)])
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    prev = None
+    for beta in (-math.inf, -1.0, 0.0, 0.5, 1.0, 2.0, math.inf):
+        dens = sa.forward(qd, kd, vd, st, beta)[2].cpu()
+        if prev is not None:
+            assert (dens <= prev).all()
+        prev = dens
+    assert (prev == 0).all()
+
+
+@pytest.mark.slow
+def test_full_size_wan_routing_exact_and_sampled_rows():
+    """75,600 tokens x 40 heads x d=128 at the benchmark's beta: every block's
+    |S_i| against the routing oracle, the output on sampled query blocks (first,
+    last partial, and random ones) of a few heads."""
+    import json
+    import os
+
+    wl = WORKLOADS["wan_75k"]
+    with open(os.path.join(os.path.dirname(__file__), "golden", "calibrated_beta.json")) as f:
+        beta = json.load(f)["wan_75k"]["beta"]
+    q, k, v = make_qkv(wl, seed=0)
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    ws = sa.workspace()
+    out, lse, dens = sa.forward(qd, kd, vd, st, beta, ws=ws)
+    assert sa.status(ws) == 0
+    dens = dens.cpu().numpy()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    nb = math.ceil(wl.N / 64)
+    for h in range(wl.H):
+        qq, kk = q[0, h].double().numpy(), k[0, h].double().numpy()
+        r = orc.route(qq, kk, beta)
+        ties = (np.abs(r["shat"] - r["tau"][:, None]) <= TIE).sum(-1)
+        _check_density(dens[0, h], r["density"], ties)
+        if h in (0, 17, 39):
+            rows = sorted({0, nb - 1, *rng.choice(nb, 6, replace=False).tolist()})
+            oo, lo, _ = orc.attend(qq, kk, v[0, h].double().numpy(), beta, rows=rows)
+            m = np.zeros(wl.N, bool)
+            for i in rows:
+                m[i * 64:min(wl.N, i * 64 + 64)] = True
+            _check_out(out[0, h], lse[0, h], oo, lo, m)
