@@ -166,10 +166,15 @@ __device__ void route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     for (int e = 0; e < VPL; ++e) q1[e] = 0.f;
   }
   const float beta = P.beta;
+  // tau_i = mu_i + beta sigma_i. sigma_i = 0 means a constant proxy row (every
+  // score equals mu_i = tau_i): nothing is strictly above it, so no block is
+  // kept, whatever rounding does to the individual scores.
   auto tau_of = [&](int i) -> float {
     if (beta == -INFINITY) return -INFINITY;
     if (beta == INFINITY) return INFINITY;
-    return P.mu[static_cast<long long>(bh) * NB + i] + beta * P.sigma[static_cast<long long>(bh) * NB + i];
+    const float sg = P.sigma[static_cast<long long>(bh) * NB + i];
+    if (sg == 0.f) return INFINITY;
+    return P.mu[static_cast<long long>(bh) * NB + i] + beta * sg;
   };
   const float tau0 = tau_of(i0);
   const float tau1 = has1 ? tau_of(i1) : INFINITY;

@@ -45,7 +45,9 @@ design notes of this repository):
  * a skipped block weighs n_j (its count of valid tokens);
  * sigma is the population standard deviation (divide by N_b); the covariance
    is computed two-pass; every block counts once whatever its n_j;
- * ties s_hat_ij == tau_i are skipped (strict ">");
+ * ties s_hat_ij == tau_i are skipped (strict ">"); a row with sigma_i = 0 is
+   constant (all its proxy scores equal mu_i = tau_i), so none of its blocks
+   is kept for finite beta;
  * beta = -inf means tau = -inf (all blocks kept, never -inf * 0); beta = +inf
    means tau = +inf (all skipped);
  * pad tokens of the last partial block are not part of any mean and are never
@@ -140,14 +142,18 @@ def row_stats(qbar: np.ndarray, kmean: np.ndarray, kcov: np.ndarray):
 # Step 5: threshold
 # --------------------------------------------------------------------------
 def thresholds(mu: np.ndarray, sigma: np.ndarray, beta: float) -> np.ndarray:
-    """tau_i = mu_i + beta sigma_i; beta = -inf / +inf give -inf / +inf."""
+    """tau_i = mu_i + beta sigma_i; beta = -inf / +inf give -inf / +inf.
+
+    A row with sigma_i = 0 is constant: every s_hat_ij equals mu_i = tau_i, so
+    under the strict ">" no block passes; its threshold is returned as +inf so
+    that rounding in s_hat cannot make a tie look like a pass."""
     if math.isnan(beta):
         raise ValueError("beta is NaN")
     if beta == -math.inf:
         return np.full(mu.shape, -math.inf)
     if beta == math.inf:
         return np.full(mu.shape, math.inf)
-    return mu + beta * sigma
+    return np.where(sigma == 0.0, math.inf, mu + beta * sigma)
 
 
 def proxy_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
