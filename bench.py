@@ -22,6 +22,7 @@ workload per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -211,6 +212,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOADS[args.workload]
+    if args.heads:
+        wl = dataclasses.replace(wl, H=args.heads)
     beta = args.beta if args.beta is not None else load_beta(args.workload)[0]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
     peaks = load_peaks()
@@ -397,6 +400,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan_75k", choices=sorted(WORKLOADS))
     ap.add_argument("--beta", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--cpu-blocks", type=int, default=24)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
