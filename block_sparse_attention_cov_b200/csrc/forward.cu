@@ -39,24 +39,45 @@
 
 namespace solattn {
 
+#ifdef SOLATTN_TRACE
+// Debug builds only: per-tile timestamps of CTA 0 (clock64), [event][index].
+__device__ unsigned long long g_trace[16][4096];
+#define SOLATTN_TRACE_EVENT(ev, idx)                                         \
+  do {                                                                       \
+    if (blockIdx.x == 0 && (idx) < 4096) g_trace[(ev)][(idx)] = clock64();   \
+  } while (0)
+#else
+#define SOLATTN_TRACE_EVENT(ev, idx) \
+  do {                               \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kBM = 128;      // rows per unit
 constexpr int kBN = 64;       // keys per tile (one block)
-constexpr int kStages = 4;    // K/V ring depth
+constexpr int kStages = 5;    // depth of the K ring and of the V ring
 constexpr int kNbMax = 4096;  // key blocks per head supported
-constexpr int kThreads = 320;
+constexpr int kThreads = 512;
+// Registers per thread after rebalancing (launched with 65536 / 512 = 128):
+// 2 softmax warpgroups x 136 + routing 120 + producer/MMA 120, times 128 threads
+// each = 65536.
+constexpr int kRegsSoftmax = 136, kRegsRouting = 120, kRegsIssue = 120;
+static_assert(128 * (2 * kRegsSoftmax + kRegsRouting + kRegsIssue) <= 65536, "register split exceeds the launch");
+constexpr int kChunk = 16;    // pooled key blocks per routing chunk (4 per routing warp)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.0f;  // log2 units a row max may grow before O is rescaled
 
-constexpr uint32_t kColQ = 0, kColO = 128, kColS = 256, kColP = 384;
+constexpr uint32_t kColQ = 0, kColS = 64, kColP = 192, kColO = 256;  // + group * 64 / 32 / 128
 
 // Wait-site ids reported in the status word when a bounded wait gives up.
 enum : uint32_t {
   kSiteRouteEmpty = 1,
   kSiteRouteFullProd,
-  kSiteKvEmpty,
+  kSiteKEmpty,
+  kSiteVEmpty,
+  kSiteMmaStall,
   kSiteRouteFullMma,
   kSiteKFull,
   kSiteSFree,
@@ -66,31 +87,46 @@ enum : uint32_t {
   kSiteRouteFullSoft,
   kSiteSFull,
   kSiteOFull,
+  kSiteRouteChunk,
+  kSiteQFree,
+  kSiteBDone,
 };
 
 template <int D>
 struct __align__(1024) Smem {
   uint8_t kt[kStages][kBN * D * 2];  // SW128 K tiles (1024-aligned: size is a multiple of 8 KB)
   uint8_t vt[kStages][kBN * D * 2];  // SW128 V tiles
+  float rchunk[2][2][kChunk][D];     // routing: [buffer][kbar | vbar][key block][column]
   uint16_t list[2][kNbMax];          // kept (union) list: j | keep-bits << 14
   float cnum[2][2][D];               // correction numerator per slot and block
   float cden[2][2];
   float cmax[2][2];                  // reference max of the correction (natural units)
   int unit[2];
   int count[2];
-  float wnum[4][2][D];               // per routing warp partial corrections
-  float wden[4][2];
-  float wmax[4][2];
+  float rscore[2][kChunk];           // proxy scores of the chunk being routed
+  float rweight[2][kChunk];          // correction weights n_j e^{s_hat - M} (0 if kept)
+  float rscale[2];                   // rescale of the running correction sums
+  float rmax[2];                     // running max of the skipped proxy scores
+  float rden[2];                     // running correction denominators
+  int rkept[2];                      // running kept counts
   uint32_t bits[2][kNbMax / 32];     // kept bitmaps of the unit being routed
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2];
-  uint64_t o_full, o_free;
+  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
+  uint64_t s_full[2], s_free[2], p_full[2], o_full[2];  // per softmax group
+  uint64_t o_free, b_done, q_free;
   uint64_t route_full[2], route_empty[2];
+  uint64_t rfull[2];                 // routing chunk buffers landed
   uint64_t mma_done;
+  float mB[2][kBM];                  // group B's final running max / sum per row, per slot
+  float lB[2][kBM];
   uint32_t tmem_base;
   int bcast;
   int abort_flag;
 };
+
+// Dynamic shared memory per CTA on sm_100 is at most 227 KB (232448 bytes);
+// one extra KB pays for the 1024-byte alignment of the TMA tiles.
+static_assert(sizeof(Smem<128>) + 1024 <= 232448, "shared memory layout too large");
+static_assert(sizeof(Smem<64>) + 1024 <= 232448, "shared memory layout too large");
 
 struct Params {
   const uint16_t* q;
@@ -114,56 +150,51 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// Routing: scores of both query blocks against every key block, kept bitmaps,
-// correction sums. 128 threads (warps 4-7), one key block per warp per trip.
+// Routing (warps 4-7, 128 threads): the pooled keys and values of the head are
+// streamed through shared memory in chunks of 32 key blocks (bulk async copies,
+// double-buffered). Per chunk: every warp scores 8 key blocks against both
+// query blocks of the unit (one float4 column slice per lane, transposed
+// butterfly reduction), the threshold test sets the kept bits, and the skipped
+// blocks' weights n_j e^{s_hat - M} are folded into per-column correction sums
+// (one column per thread). The proxy row never leaves shared memory.
 // ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void corr_add(float& M, float& den, float (&num)[D / 32], float sh, float nj,
-                                         const float (&vv)[D / 32]) {
-  if (sh > M) {
-    const float sc = ex2_approx((M - sh) * kLog2e);  // 0 when M = -inf
-    den *= sc;
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) num[e] *= sc;
-    M = sh;
-  }
-  const float w = nj * ex2_approx((sh - M) * kLog2e);
-  den += w;
-#pragma unroll
-  for (int e = 0; e < D / 32; ++e) num[e] = fmaf(w, vv[e], num[e]);
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
+// Returns false if a bounded wait gave up (the CTA is aborting).
 template <int D>
-__device__ __forceinline__ void load_vec(const float* p, float (&x)[D / 32]) {
-  if constexpr (D == 128) {
-    const float4 t = __ldg(reinterpret_cast<const float4*>(p));
-    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
-  } else {
-    const float2 t = __ldg(reinterpret_cast<const float2*>(p));
-    x[0] = t.x; x[1] = t.y;
-  }
-}
-
-template <int D>
-__device__ void route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair, int rt) {
-  constexpr int VPL = D / 32;
+__device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair, int rt, uint32_t& chunk_ctr,
+                           volatile int* abort_flag, DeviceStatus* st, int u) {
+  constexpr int VPL = D / 32;  // columns per lane in the scoring layout
   const int rw = rt / 32, lane = rt % 32;
   const int NB = P.NB;
   const int i0 = 2 * pair, i1 = 2 * pair + 1;
   const bool has1 = i1 < NB;
-  const int nwords = (NB + 31) / 32;
-  for (int w = rt; w < nwords; w += 128) {
-    sm.bits[0][w] = 0u;
-    sm.bits[1][w] = 0u;
-  }
+  const int nchunks = (NB + kChunk - 1) / kChunk;
+  const float* kb = P.kbar + static_cast<long long>(bh) * NB * D;
+  const float* vb = P.vbar + static_cast<long long>(bh) * NB * D;
+  auto issue = [&](int c) {
+    const int j0 = c * kChunk;
+    const int nk = min(kChunk, NB - j0);
+    const uint32_t buf = (chunk_ctr + c) & 1;
+    const uint32_t bytes = static_cast<uint32_t>(nk) * D * 4;
+    mbar_arrive_expect_tx(&sm.rfull[buf], 2 * bytes);
+    bulk_copy_g2s(&sm.rchunk[buf][0][0][0], kb + static_cast<long long>(j0) * D, bytes, &sm.rfull[buf]);
+    bulk_copy_g2s(&sm.rchunk[buf][1][0][0], vb + static_cast<long long>(j0) * D, bytes, &sm.rfull[buf]);
+  };
+  if (rt == 0) issue(0);
+
   const float* qb = P.qbar + static_cast<long long>(bh) * NB * D;
   float q0[VPL], q1[VPL];
-  load_vec<D>(qb + static_cast<long long>(i0) * D + lane * VPL, q0);
-  if (has1) {
-    load_vec<D>(qb + static_cast<long long>(i1) * D + lane * VPL, q1);
-  } else {
 #pragma unroll
-    for (int e = 0; e < VPL; ++e) q1[e] = 0.f;
+  for (int e = 0; e < VPL; ++e) {
+    q0[e] = qb[static_cast<long long>(i0) * D + lane * VPL + e];
+    q1[e] = has1 ? qb[static_cast<long long>(i1) * D + lane * VPL + e] : 0.f;
   }
   const float beta = P.beta;
   // tau_i = mu_i + beta sigma_i. sigma_i = 0 means a constant proxy row (every
@@ -180,101 +211,166 @@ __device__ void route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   const float tau1 = has1 ? tau_of(i1) : INFINITY;
   const float scale = rsqrtf(static_cast<float>(D));
   const int nlast = P.N - (NB - 1) * kBN;
-  named_bar_sync(1, 128);  // bitmaps cleared
+  if (rt < 2) {
+    sm.rmax[rt] = -INFINITY;
+    sm.rden[rt] = 0.f;
+    sm.rkept[rt] = 0;
+  }
+  // correction accumulators: thread rt owns column rt (D = 128: both blocks;
+  // D = 64: block rt / 64, column rt % 64)
+  constexpr int NACC = D / 64;
+  float acc[NACC];
+#pragma unroll
+  for (int a = 0; a < NACC; ++a) acc[a] = 0.f;
 
-  float M0 = -INFINITY, M1 = -INFINITY, den0 = 0.f, den1 = 0.f;
-  float num0[VPL], num1[VPL];
+  bool ok = true;
+  for (int c = 0; c < nchunks; ++c) {
+    const uint32_t g = chunk_ctr + c, buf = g & 1;
+    if (rt == 0 && c + 1 < nchunks) issue(c + 1);  // buffer (c+1)&1 was released by chunk c-1
+    const bool landed = mbar_wait(&sm.rfull[buf], (g >> 1) & 1, abort_flag, st, kSiteRouteChunk, u);
+    if (named_bar_or(1, 128, !landed || *abort_flag)) {
+      // aborting: let the copies already issued (chunks c and c + 1) land first
+      if (rt == 0) {
+        mbar_wait_quiet(&sm.rfull[buf], (g >> 1) & 1);
+        if (c + 1 < nchunks) mbar_wait_quiet(&sm.rfull[(g + 1) & 1], ((g + 1) >> 1) & 1);
+      }
+      ok = false;
+      break;
+    }
+    const int j0 = c * kChunk;
+    const int nk = min(kChunk, NB - j0);
+    // ---- scores: warp rw handles key blocks 4 rw .. 4 rw + 3 of the chunk
+    float v[8];
 #pragma unroll
-  for (int e = 0; e < VPL; ++e) num0[e] = num1[e] = 0.f;
-  const float* kb = P.kbar + static_cast<long long>(bh) * NB * D + lane * VPL;
-  const float* vb = P.vbar + static_cast<long long>(bh) * NB * D + lane * VPL;
-  for (int j = rw; j < NB; j += 4) {
-    float kv[VPL];
-    load_vec<D>(kb + static_cast<long long>(j) * D, kv);
-    float d0 = 0.f, d1 = 0.f;
+    for (int kk = 0; kk < 4; ++kk) {
+      const float* row = &sm.rchunk[buf][0][rw * 4 + kk][lane * VPL];
+      float x[VPL];
+      if constexpr (VPL == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(row);
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(row);
+        x[0] = t.x; x[1] = t.y;
+      }
+      float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < VPL; ++e) {
-      d0 = fmaf(q0[e], kv[e], d0);
-      d1 = fmaf(q1[e], kv[e], d1);
+      for (int e = 0; e < VPL; ++e) {
+        d0 = fmaf(q0[e], x[e], d0);
+        d1 = fmaf(q1[e], x[e], d1);
+      }
+      v[2 * kk] = d0;
+      v[2 * kk + 1] = d1;
+    }
+    // transposed butterfly: after it, lane l holds the full sum of value (l >> 2)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool up = lane & 16;
+      const float send = up ? v[i] : v[4 + i];
+      const float keep = up ? v[4 + i] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      d0 += __shfl_xor_sync(0xffffffffu, d0, off);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, off);
+    for (int i = 0; i < 2; ++i) {
+      const bool up = lane & 8;
+      const float send = up ? v[i] : v[2 + i];
+      const float keep = up ? v[2 + i] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
     }
-    const float sh0 = d0 * scale, sh1 = d1 * scale;
-    const bool k0 = sh0 > tau0;
-    const bool k1 = has1 && (sh1 > tau1);
-    if (lane == 0) {
-      if (k0) atomicOr(&sm.bits[0][j >> 5], 1u << (j & 31));
-      if (k1) atomicOr(&sm.bits[1][j >> 5], 1u << (j & 31));
+    {
+      const bool up = lane & 4;
+      const float send = up ? v[0] : v[1];
+      const float keep = up ? v[1] : v[0];
+      v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
     }
-    const bool c0 = !k0, c1 = has1 && !k1;
-    if (c0 || c1) {
-      float vv[VPL];
-      load_vec<D>(vb + static_cast<long long>(j) * D, vv);
-      const float nj = static_cast<float>(j == NB - 1 ? nlast : kBN);
-      if (c0) corr_add<D>(M0, den0, num0, sh0, nj, vv);
-      if (c1) corr_add<D>(M1, den1, num1, sh1, nj, vv);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+    if ((lane & 3) == 0) {
+      const int idx = lane >> 2;  // = 2 * kk + block
+      sm.rscore[idx & 1][rw * 4 + (idx >> 1)] = v[0] * scale;
     }
+    named_bar_sync(1, 128);
+    // ---- threshold, kept bits, correction weights (warp 0: block 0, warp 1: block 1)
+    if (rw < 2) {
+      const int b = rw;
+      const bool valid = lane < nk && (b == 0 || has1);
+      const float sh = sm.rscore[b][lane & (kChunk - 1)];
+      const bool kept = valid && sh > (b == 0 ? tau0 : tau1);
+      const bool skip = valid && !kept;
+      const uint32_t kmask = __ballot_sync(0xffffffffu, kept);
+      float mx = skip ? sh : -INFINITY;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mold = sm.rmax[b];
+      const float mnew = fmaxf(mold, mx);
+      const float nj = static_cast<float>(j0 + lane == NB - 1 ? nlast : kBN);
+      const float w = skip ? nj * ex2_approx((sh - mnew) * kLog2e) : 0.f;
+      float wsum = w;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+      if (lane < kChunk) sm.rweight[b][lane] = w;
+      if (lane == 0) {
+        const float sc = (mold == -INFINITY) ? 0.f : ex2_approx((mold - mnew) * kLog2e);
+        sm.rscale[b] = sc;
+        sm.rden[b] = sm.rden[b] * sc + wsum;
+        sm.rmax[b] = mnew;
+        sm.rkept[b] += __popc(kmask);
+        // two 16-block chunks per 32-bit bitmap word (even chunk first)
+        if (c & 1) sm.bits[b][c >> 1] |= kmask << 16;
+        else sm.bits[b][c >> 1] = kmask;
+      }
+    }
+    named_bar_sync(1, 128);
+    // ---- correction sums: sum_j w_bj vbar_j[col]
+    {
+      const float* vrows = &sm.rchunk[buf][1][0][0];
+      if constexpr (D == 128) {
+        const float sc0 = sm.rscale[0], sc1 = sm.rscale[1];
+        float a0 = acc[0] * sc0, a1 = acc[1] * sc1;
+        for (int jj = 0; jj < nk; ++jj) {
+          const float x = vrows[jj * D + rt];
+          a0 = fmaf(sm.rweight[0][jj], x, a0);
+          a1 = fmaf(sm.rweight[1][jj], x, a1);
+        }
+        acc[0] = a0;
+        acc[1] = a1;
+      } else {
+        const int b = rt / 64, col = rt % 64;
+        float a0 = acc[0] * sm.rscale[b];
+        for (int jj = 0; jj < nk; ++jj) a0 = fmaf(sm.rweight[b][jj], vrows[jj * D + col], a0);
+        acc[0] = a0;
+      }
+    }
+    named_bar_sync(1, 128);  // chunk buffer and scratch free again
   }
-  // per-warp partials -> shared
-#pragma unroll
-  for (int e = 0; e < VPL; ++e) {
-    sm.wnum[rw][0][lane * VPL + e] = num0[e];
-    sm.wnum[rw][1][lane * VPL + e] = num1[e];
-  }
-  if (lane == 0) {
-    sm.wden[rw][0] = den0;
-    sm.wden[rw][1] = den1;
-    sm.wmax[rw][0] = M0;
-    sm.wmax[rw][1] = M1;
-  }
-  named_bar_sync(1, 128);
-  // combine the four warps (fixed order)
-  for (int idx = rt; idx < 2 * D; idx += 128) {
-    const int b = idx / D, e = idx % D;
-    float Mb = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) Mb = fmaxf(Mb, sm.wmax[w][b]);
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float mw = sm.wmax[w][b];
-      if (mw != -INFINITY) acc = fmaf(sm.wnum[w][b][e], ex2_approx((mw - Mb) * kLog2e), acc);
-    }
-    sm.cnum[s][b][e] = acc;
+  chunk_ctr += nchunks;
+  if (!ok) return false;
+  // ---- publish the unit's correction and kept list into slot s
+  if constexpr (D == 128) {
+    sm.cnum[s][0][rt] = acc[0];
+    sm.cnum[s][1][rt] = acc[1];
+  } else {
+    sm.cnum[s][rt / 64][rt % 64] = acc[0];
   }
   if (rt < 2) {
-    const int b = rt;
-    float Mb = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) Mb = fmaxf(Mb, sm.wmax[w][b]);
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float mw = sm.wmax[w][b];
-      if (mw != -INFINITY) acc = fmaf(sm.wden[w][b], ex2_approx((mw - Mb) * kLog2e), acc);
-    }
-    sm.cden[s][b] = acc;
-    sm.cmax[s][b] = Mb;
+    sm.cden[s][rt] = sm.rden[rt];
+    sm.cmax[s][rt] = sm.rmax[rt];
   }
-  // ordered union list from the bitmaps (warp 0 of the routing group)
   if (rw == 0) {
-    int base = 0, kept0 = 0, kept1 = 0;
+    const int nwords = (nchunks + 1) / 2;  // one 32-bit word per two chunks
+    int base = 0;
     for (int w0 = 0; w0 < nwords; w0 += 32) {
       const int wi = w0 + lane;
       const uint32_t m0 = wi < nwords ? sm.bits[0][wi] : 0u;
       const uint32_t m1 = wi < nwords ? sm.bits[1][wi] : 0u;
       uint32_t un = m0 | m1;
-      const int c = __popc(un);
-      int incl = c;
+      const int cnt = __popc(un);
+      int incl = cnt;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += y;
       }
-      int pos = base + incl - c;
+      int pos = base + incl - cnt;
       while (un) {
         const int bit = __ffs(un) - 1;
         const uint32_t flags = ((m0 >> bit) & 1u) | (((m1 >> bit) & 1u) << 1);
@@ -282,47 +378,136 @@ __device__ void route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
         un &= un - 1u;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
-      kept0 += __popc(m0);
-      kept1 += __popc(m1);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      kept0 += __shfl_xor_sync(0xffffffffu, kept0, off);
-      kept1 += __shfl_xor_sync(0xffffffffu, kept1, off);
     }
     if (lane == 0) {
       sm.count[s] = base;
       if (P.density) {
-        P.density[static_cast<long long>(bh) * NB + i0] = kept0;
-        if (has1) P.density[static_cast<long long>(bh) * NB + i1] = kept1;
+        P.density[static_cast<long long>(bh) * NB + i0] = sm.rkept[0];
+        if (has1) P.density[static_cast<long long>(bh) * NB + i1] = sm.rkept[1];
       }
     }
   }
+  return true;
 }
 
-// Copies the unit's 128 Q rows (bf16 pairs, one 32-bit TMEM column per pair)
-// into the Q slot; rows past N are zero.
+// Reads the unit's 128 Q rows (bf16 pairs = one 32-bit TMEM column per pair)
+// into registers; rows past N are zero.
 template <int D>
-__device__ __forceinline__ void load_q_to_tmem(const Params& P, uint32_t tmem, int s, int bh, int pair, int rt) {
+__device__ __forceinline__ void load_q_rows(const Params& P, int bh, int pair, int rt, uint32_t (&w)[D / 2]) {
   const int row = pair * kBM + rt;
-  const uint32_t taddr = tmem + (static_cast<uint32_t>((rt / 32) * 32) << 16) + kColQ + s * 64;
   const uint4* src = reinterpret_cast<const uint4*>(P.q + (static_cast<long long>(bh) * P.N + row) * D);
   const bool ok = row < P.N;
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) {
-    uint32_t w[32];
+  for (int x = 0; x < D / 8; ++x) {
+    const uint4 t = ok ? __ldg(src + x) : make_uint4(0, 0, 0, 0);
+    w[4 * x] = t.x; w[4 * x + 1] = t.y; w[4 * x + 2] = t.z; w[4 * x + 3] = t.w;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_q_tmem(uint32_t tmem, int rt, const uint32_t (&w)[D / 2]) {
+  const uint32_t taddr = tmem + (static_cast<uint32_t>((rt / 32) * 32) << 16) + kColQ;
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const uint4 t = ok ? __ldg(src + c * 8 + x) : make_uint4(0, 0, 0, 0);
-      w[4 * x] = t.x; w[4 * x + 1] = t.y; w[4 * x + 2] = t.z; w[4 * x + 3] = t.w;
-    }
-    tmem_st32(taddr + c * 32, w);
+  for (int c = 0; c < D / 64; ++c) {
+    uint32_t x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = w[c * 32 + e];
+    tmem_st32(taddr + c * 32, x);
   }
   tmem_wait_st();
 }
 
 // ---------------------------------------------------------------------------
-// The kernel
+// Softmax arithmetic of one row and one 64-key tile (log2 domain, lazily
+// rescaled running max m, running sum l). sv/sw hold S columns 0-31 / 32-63,
+// nv = valid keys of the tile. Writes the bf16 P row into pw; returns whether
+// the row's O must be multiplied by `rescale` before this tile's PV.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2_from_bits(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Masks the pad keys of a partial tile and folds the tile's row max into the
+// lazily rescaled running max m (log2 units). Returns whether the row's O and
+// l must be multiplied by `rescale` (= 2^(m_old - m_new)) before this tile.
+__device__ __forceinline__ bool softmax_max(uint32_t (&sv)[32], uint32_t (&sw)[32], int nv, float sl2, float& m,
+                                            float& rescale) {
+  constexpr uint32_t kNegInf = 0xFF800000u;
+  if (nv < 64) {  // only the last key block of a head can be partial
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      if (c >= nv) sv[c] = kNegInf;
+      if (c + 32 >= nv) sw[c] = kNegInf;
+    }
+  }
+  float t[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    t[i] = fmax3(fmax3(__uint_as_float(sv[8 * i]), __uint_as_float(sv[8 * i + 1]), __uint_as_float(sv[8 * i + 2])),
+                 fmax3(__uint_as_float(sv[8 * i + 3]), __uint_as_float(sv[8 * i + 4]), __uint_as_float(sv[8 * i + 5])),
+                 fmaxf(__uint_as_float(sv[8 * i + 6]), __uint_as_float(sv[8 * i + 7])));
+    t[4 + i] = fmax3(fmax3(__uint_as_float(sw[8 * i]), __uint_as_float(sw[8 * i + 1]), __uint_as_float(sw[8 * i + 2])),
+                     fmax3(__uint_as_float(sw[8 * i + 3]), __uint_as_float(sw[8 * i + 4]), __uint_as_float(sw[8 * i + 5])),
+                     fmaxf(__uint_as_float(sw[8 * i + 6]), __uint_as_float(sw[8 * i + 7])));
+  }
+  const float mx = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(fmax3(t[3], t[4], t[5]), t[6], t[7])) * sl2;
+  rescale = 1.f;
+  if (mx > m + kRescaleSlack) {
+    const bool need = m != -INFINITY;
+    if (need) rescale = ex2_approx(m - mx);
+    m = mx;
+    return need;
+  }
+  return false;
+}
+
+// P for 16 consecutive columns (x holds their raw S bits): 8 packed bf16x2
+// words; adds the fp32 probabilities to l.
+__device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, uint64_t nm2, float& l,
+                                              uint32_t (&pw)[8]) {
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; c += 2) {
+    float y0, y1;
+    f2_split(ffma2(f2_from_bits(x[c], x[c + 1]), sc2, nm2), y0, y1);
+    const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);  // ex2(-inf) = 0 for masked keys
+    if (c & 2) a1 += p0 + p1; else a0 += p0 + p1;
+    pw[c >> 1] = pack_bf16x2(p0, p1);
+  }
+  l += a0 + a1;
+}
+
+// ---------------------------------------------------------------------------
+// The kernel. 512 threads = 16 warps:
+//   warps 0-3   softmax group A (even global tiles) + epilogue
+//   warps 4-7   softmax group B (odd global tiles)
+//   warps 8-11  routing, one unit ahead (Q rows into TMEM after the previous
+//               unit's last QK has completed)
+//   warp 12     TMA producer of the K tiles of the kept list
+//   warp 13     MMA issuer (event loop, one elected lane issues)
+//   warp 14     TMA producer of the V tiles
+//   warp 15     idle (completes the last warpgroup for register rebalancing)
+// TMEM: Q at 0 (64 columns), S_A/S_B at 64/128, P_A/P_B at 192/224,
+// O_A/O_B at 256/384. Each group keeps its own running max, sum and O; the
+// epilogue merges the two with the skipped-block correction.
 // ---------------------------------------------------------------------------
 template <int D, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -339,26 +524,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.k_full[i], 1);
       mbar_init(&sm.v_full[i], 1);
-      mbar_init(&sm.kv_empty[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_free[i], 4);
       mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.route_full[i], 1);
-      mbar_init(&sm.route_empty[i], 6);
+      mbar_init(&sm.route_empty[i], 11);  // 2 producers + MMA + 8 softmax warps
+      mbar_init(&sm.rfull[i], 1);
     }
-    mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_free, 4);
+    mbar_init(&sm.b_done, 4);
+    mbar_init(&sm.q_free, 1);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
@@ -366,19 +555,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp >= 12) {
+    regs_dec<kRegsIssue>();
+  } else if (warp >= 8) {
+    regs_dec<kRegsRouting>();
+  } else {
+    regs_inc<kRegsSoftmax>();
+  }
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < 12) {
     // ======================= routing =======================
-    const int rt = tid - 128;
+    const int rt = tid - 256;
+    uint32_t chunk_ctr = 0;  // routing chunks consumed so far (buffer parity)
     for (int n = 0;; ++n) {
       const int s = n & 1;
       if (n >= 2) {
-        if (rt == 0)
-          sm.bcast = mbar_wait(&sm.route_empty[s], ((n >> 1) - 1) & 1, abort_flag, st, kSiteRouteEmpty, 0) ? 1 : 0;
-        named_bar_sync(1, 128);
-        const int ok = sm.bcast;
-        named_bar_sync(1, 128);
-        if (!ok) break;
+        bool okw = true;
+        if (rt == 0) okw = mbar_wait(&sm.route_empty[s], ((n >> 1) - 1) & 1, abort_flag, st, kSiteRouteEmpty, 0);
+        if (named_bar_or(1, 128, !okw)) break;
       }
       if (rt == 0) sm.bcast = static_cast<int>(atomicAdd(&st->tile_counter, 1u));
       named_bar_sync(1, 128);
@@ -393,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int bh = u / P.npairs, pair = u % P.npairs;
-      load_q_to_tmem<D>(P, tmem, s, bh, pair, rt);
+      SOLATTN_TRACE_EVENT(13, rt == 0 ? n : 4096);
       if constexpr (ROUTE) {
-        route_unit<D>(sm, P, s, bh, pair, rt);
+        if (!route_unit<D>(sm, P, s, bh, pair, rt, chunk_ctr, abort_flag, st, u)) break;
       } else {
         if (rt == 0) {
           sm.count[s] = P.NB;
@@ -403,15 +597,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.cmax[s][0] = sm.cmax[s][1] = -INFINITY;
         }
       }
+      uint32_t qw[D / 2];
+      load_q_rows<D>(P, bh, pair, rt, qw);
+      if (n >= 1) {  // the Q slot is free once every QK of the previous unit has completed
+        const bool okq = mbar_wait(&sm.q_free, (n - 1) & 1, abort_flag, st, kSiteQFree, u);
+        if (named_bar_or(1, 128, !okq)) break;
+      }
+      tc_fence_after();
+      store_q_tmem<D>(tmem, rt, qw);
       tc_fence_before();
       named_bar_sync(1, 128);
       if (rt == 0) {
         sm.unit[s] = u;
         mbar_arrive(&sm.route_full[s]);
+        SOLATTN_TRACE_EVENT(14, n);
       }
     }
-  } else if (warp == 8) {
-    // ======================= TMA producer (lane 0 issues) =======================
+  } else if (warp == 12 || warp == 14) {
+    // ======================= TMA producers: warp 12 = K tiles, warp 14 = V tiles =======================
+    const bool isK = warp == 12;
+    uint64_t* full = isK ? sm.k_full : sm.v_full;
+    uint64_t* empty = isK ? sm.k_empty : sm.v_empty;
+    const CUtensorMap* map = isK ? &tmK : &tmV;
+    uint8_t* ring = isK ? &sm.kt[0][0] : &sm.vt[0][0];
     uint32_t g = 0;
     for (int n = 0;; ++n) {
       const int s = n & 1;
@@ -424,37 +632,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (; t < T; ++t) {
         const int j = ROUTE ? (sm.list[s][t] & 0x3FFF) : t;
         const uint32_t gt = g + t, stg = gt % kStages, r = gt / kStages;
-        if (r >= 1 && !warp_wait(&sm.kv_empty[stg], (r - 1) & 1, abort_flag, st, kSiteKvEmpty, u)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.k_full[stg], kBN * D * 2);
+        if (r >= 1 && !warp_wait(&empty[stg], (r - 1) & 1, abort_flag, st, isK ? kSiteKEmpty : kSiteVEmpty, u)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full[stg], kBN * D * 2);
 #pragma unroll
           for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(&sm.kt[stg][pnl * 8192], &tmK, &sm.k_full[stg], pnl * 64, j * kBN, bh);
-          mbar_arrive_expect_tx(&sm.v_full[stg], kBN * D * 2);
-#pragma unroll
-          for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(&sm.vt[stg][pnl * 8192], &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh);
+            tma_load_3d(ring + stg * (kBN * D * 2) + pnl * 8192, map, &full[stg], pnl * 64, j * kBN, bh);
         }
         __syncwarp();
       }
       g += t;
       if (t < T) break;  // aborted
-      if (lane == 0) mbar_arrive(&sm.route_empty[s]);
+      if (elect_one()) mbar_arrive(&sm.route_empty[s]);
       __syncwarp();
     }
-    // teardown: let every issued copy land before the CTA exits
-    if (lane == 0) {
+    if (lane == 0) {  // teardown: every issued copy lands before the CTA exits
       const uint32_t first = g > static_cast<uint32_t>(kStages) ? g - kStages : 0u;
-      for (uint32_t gt = first; gt < g; ++gt) {
-        mbar_wait_quiet(&sm.k_full[gt % kStages], (gt / kStages) & 1);
-        mbar_wait_quiet(&sm.v_full[gt % kStages], (gt / kStages) & 1);
-      }
+      for (uint32_t gt = first; gt < g; ++gt) mbar_wait_quiet(&full[gt % kStages], (gt / kStages) & 1);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ======================= MMA issuer (lane 0 issues) =======================
+  } else if (warp == 15) {
+    // idle warp (completes the last warpgroup)
+  } else if (warp == 13) {
+    // ======================= MMA issuer =======================
+    // Event loop: issues QK of the next tile whose K tile has landed and whose
+    // S buffer its group has read, and PV of the next tile whose P is ready,
+    // whichever is ready first (QKs in tile order, PVs in tile order).
     constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
+    constexpr uint32_t kTileBytes = kBN * D * 2;
+    const uint64_t kdesc0 = sw128_desc(smem_u32(&sm.kt[0][0]), 16, 1024);
+    const uint64_t vdesc0 = sw128_desc(smem_u32(&sm.vt[0][0]), 8192, 1024);
     uint32_t g = 0;
     bool ok = true;
     for (int n = 0; ok; ++n) {
@@ -464,62 +672,98 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      const uint32_t qaddr = tmem + kColQ + s * 64;
-      for (int t = 0; t <= T; ++t) {
-        if (t < T) {
-          const uint32_t gt = g + t, stg = gt % kStages, b = gt & 1, use = gt >> 1;
-          if (!warp_wait(&sm.k_full[stg], (gt / kStages) & 1, abort_flag, st, kSiteKFull, u)) { ok = false; break; }
-          if (use >= 1 && !warp_wait(&sm.s_free[b], (use - 1) & 1, abort_flag, st, kSiteSFree, u)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t kaddr = smem_u32(&sm.kt[stg][0]);
+      if (T == 0) {
+        if (elect_one()) mma_commit(&sm.q_free);
+        __syncwarp();
+        if (n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) break;
+      }
+      int nq = 0, np = 0;
+      bool ofree_seen = n == 0;
+      uint32_t first_pv = 3u;  // bit w: group w has not accumulated into its O in this unit
+      unsigned long long t_idle = 0;
+      while (np < T) {
+        bool progressed = false;
+        if (np < nq) {
+          const uint32_t gp = g + np, stp = gp % kStages, w = gp & 1, usep = gp >> 1;
+          if (!ofree_seen) ofree_seen = __all_sync(0xffffffffu, mbar_test(&sm.o_free, (n - 1) & 1));
+          if (ofree_seen && __all_sync(0xffffffffu, mbar_test(&sm.p_full[w], usep & 1) &&
+                                                         mbar_test(&sm.v_full[stp], (gp / kStages) & 1))) {
+            tc_fence_after();
+            if (elect_one()) {
+              SOLATTN_TRACE_EVENT(11, gp);
+              const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
+              const uint32_t acc0 = (first_pv >> w) & 1u ? 0u : 1u;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t bdesc = sw128_desc(kaddr + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
-              mma_ts(tmem + kColS + b * 64, qaddr + kk * 8, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ts(tmem + kColO + w * 128, tmem + kColP + w * 32 + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                       kk > 0 ? 1u : acc0);
+              mma_commit(&sm.v_empty[stp]);
+              mma_commit(&sm.o_full[w]);
             }
-            mma_commit(&sm.s_full[b]);
+            __syncwarp();
+            first_pv &= ~(1u << w);
+            ++np;
+            progressed = true;
           }
-          __syncwarp();
         }
-        if (t >= 1) {
-          const int tp = t - 1;
-          const uint32_t gp = g + tp, stp = gp % kStages, bp = gp & 1, usep = gp >> 1;
-          if (tp == 0 && n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) { ok = false; break; }
-          if (!warp_wait(&sm.p_full[bp], usep & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
-          if (!warp_wait(&sm.v_full[stp], (gp / kStages) & 1, abort_flag, st, kSiteVFull, u)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t vaddr = smem_u32(&sm.vt[stp][0]);
+        if (nq < T) {
+          const uint32_t gt = g + nq, stg = gt % kStages, w = gt & 1, use = gt >> 1;
+          if (__all_sync(0xffffffffu, mbar_test(&sm.k_full[stg], (gt / kStages) & 1) &&
+                                          (use == 0 || mbar_test(&sm.s_free[w], (use - 1) & 1)))) {
+            tc_fence_after();
+            if (elect_one()) {
+              const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              const uint64_t bdesc = sw128_desc(vaddr + kk * 2048, 8192, 1024);
-              mma_ts(tmem + kColO, tmem + kColP + bp * 32 + kk * 8, bdesc, idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_ts(tmem + kColS + w * 64, tmem + kColQ + kk * 8,
+                       kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+              mma_commit(&sm.s_full[w]);
+              mma_commit(&sm.k_empty[stg]);
+              if (nq == T - 1) mma_commit(&sm.q_free);
+              SOLATTN_TRACE_EVENT(10, gt);
             }
-            mma_commit(&sm.kv_empty[stp]);
-            mma_commit(&sm.o_full);
+            __syncwarp();
+            ++nq;
+            progressed = true;
           }
-          __syncwarp();
+        }
+        if (progressed) {
+          t_idle = 0;
+        } else {  // bounded: give up if nothing became ready for the wait budget
+          const unsigned long long now = global_timer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitBudgetNs || *abort_flag) {
+            if (lane == 0 && !*abort_flag && atomicCAS(&st->error, 0u, kErrTimeout) == 0u) {
+              st->where = kSiteMmaStall;
+              st->unit = static_cast<uint32_t>(u);
+            }
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
         }
       }
       if (!ok) break;
-      if (T == 0 && n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) break;
-      if (lane == 0) mma_commit(&sm.route_empty[s]);
+      if (elect_one()) mma_commit(&sm.route_empty[s]);
       __syncwarp();
       g += T;
     }
-    // teardown: every issued MMA completes before TMEM is released
-    if (lane == 0) mma_commit(&sm.mma_done);
+    if (elect_one()) mma_commit(&sm.mma_done);  // teardown: issued MMAs complete before TMEM is freed
     __syncwarp();
     mbar_wait_quiet(&sm.mma_done, 0);
     __syncwarp();
   } else {
-    // ======================= softmax + epilogue (warps 0-3) =======================
-    const int r = tid;           // row of the unit == TMEM lane
+    // ======================= softmax groups A (warps 0-3) and B (4-7) =======================
+    const int grp = warp >> 2;   // 0 = A (even global tiles), 1 = B (odd)
+    const int r = tid & 127;     // row of the unit == TMEM lane
     const int blk = r >> 6;      // which of the two query blocks
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = kLog2e * rsqrtf(static_cast<float>(D));
     const int nlast = P.N - (P.NB - 1) * kBN;
+    const uint32_t colS = tmem + kColS + grp * 64 + lane_off;
+    const uint32_t colP = tmem + kColP + grp * 32 + lane_off;
+    const uint32_t colO = tmem + kColO + grp * 128 + lane_off;
     uint32_t g = 0;
     for (int n = 0;; ++n) {
       const int s = n & 1;
@@ -530,124 +774,135 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int T = sm.count[s];
       const int bh = u / P.npairs, pair = u % P.npairs;
       float m = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int t = 0; t < T; ++t) {
-        const uint32_t gt = g + t, b = gt & 1, use = gt >> 1;
+      bool ok = true, first = true;
+      uint32_t last_use = 0;
+      for (int t = ((g & 1u) == static_cast<uint32_t>(grp)) ? 0 : 1; t < T; t += 2) {
+        const uint32_t gt = g + t, use = gt >> 1;
         const uint32_t entry = ROUTE ? sm.list[s][t] : (static_cast<uint32_t>(t) | 0xC000u);
         const int j = entry & 0x3FFF;
         const bool mine = (entry >> (14 + blk)) & 1u;  // warp-uniform
-        if (!warp_wait(&sm.s_full[b], use & 1, abort_flag, st, kSiteSFull, u)) { ok = false; break; }
+        if (!warp_wait(&sm.s_full[grp], use & 1, abort_flag, st, kSiteSFull, u)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[32], sw[32];  // S columns 0-31 and 32-63 of this row
+        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 0, gt);
+        uint32_t sv[32], sw[32];
         if (mine) {
-          tmem_ld32(tmem + kColS + b * 64 + lane_off, sv);
-          tmem_ld32(tmem + kColS + b * 64 + 32 + lane_off, sw);
+          tmem_ld32(colS, sv);
+          tmem_ld32(colS + 32, sw);
           tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free[b]);
-        uint32_t pw[32];
+        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 1, gt);
+        if (lane == 0) mbar_arrive(&sm.s_free[grp]);
         float rescale = 1.f;
         bool need = false;
-        if (mine) {
-          const int nv = (j == P.NB - 1) ? nlast : kBN;
-          float mx = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            mx = fmaxf(mx, c < nv ? __uint_as_float(sv[c]) : -INFINITY);
-            mx = fmaxf(mx, c + 32 < nv ? __uint_as_float(sw[c]) : -INFINITY);
-          }
-          mx *= sl2;
-          if (mx > m + kRescaleSlack) {
-            if (m != -INFINITY) {
-              need = true;
-              rescale = ex2_approx(m - mx);
-              l *= rescale;
-            }
-            m = mx;
-          }
-          float sum = 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = c < nv ? ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -m)) : 0.f;
-            const float p1 = c + 1 < nv ? ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -m)) : 0.f;
-            const float p2 = c + 32 < nv ? ex2_approx(fmaf(__uint_as_float(sw[c]), sl2, -m)) : 0.f;
-            const float p3 = c + 33 < nv ? ex2_approx(fmaf(__uint_as_float(sw[c + 1]), sl2, -m)) : 0.f;
-            sum += (p0 + p1) + (p2 + p3);
-            pw[c / 2] = pack_bf16x2(p0, p1);
-            pw[16 + c / 2] = pack_bf16x2(p2, p3);
-          }
-          l += sum;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pw[c] = 0u;
-        }
-        // PV of the previous tile must be complete: its P buffer and O are touched next
-        if (t >= 1 && !warp_wait(&sm.o_full, (gt - 1) & 1, abort_flag, st, kSiteOFull, u)) { ok = false; break; }
+        if (mine) need = softmax_max(sv, sw, (j == P.NB - 1) ? nlast : kBN, sl2, m, rescale);
+        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 2, gt);
+        // this group's previous PV must be complete: it read P and wrote O
+        if (!first && !warp_wait(&sm.o_full[grp], (use - 1) & 1, abort_flag, st, kSiteOFull, u)) { ok = false; break; }
         tc_fence_after();
+        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 3, gt);
         if (__any_sync(0xffffffffu, need)) {
+          l *= rescale;
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t ov[32];
-            tmem_ld32(tmem + kColO + ch * 32 + lane_off, ov);
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t ov[16];
+            tmem_ld16(colO + ch * 16, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * rescale);
-            tmem_st32(tmem + kColO + ch * 32 + lane_off, ov);
+            for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * rescale);
+            tmem_st16(colO + ch * 16, ov);
           }
         }
-        tmem_st32(tmem + kColP + b * 32 + lane_off, pw);
+        if (mine) {
+          const uint64_t sc2 = f2_from_bits(__float_as_uint(sl2), __float_as_uint(sl2));
+          const uint64_t nm2 = f2_from_bits(__float_as_uint(-m), __float_as_uint(-m));
+          uint32_t pw[8];
+          softmax_slice(&sv[0], sc2, nm2, l, pw);
+          tmem_st8(colP, pw);
+          softmax_slice(&sv[16], sc2, nm2, l, pw);
+          tmem_st8(colP + 8, pw);
+          softmax_slice(&sw[0], sc2, nm2, l, pw);
+          tmem_st8(colP + 16, pw);
+          softmax_slice(&sw[16], sc2, nm2, l, pw);
+          tmem_st8(colP + 24, pw);
+        } else {
+          uint32_t z[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) z[c] = 0u;
+          tmem_st16(colP, z);
+          tmem_st16(colP + 16, z);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[b]);
+        if (lane == 0) mbar_arrive(&sm.p_full[grp]);
+        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 4, gt);
+        first = false;
+        last_use = use;
       }
       if (!ok) break;
-      // ---------------- epilogue ----------------
-      if (T >= 1) {
-        if (!warp_wait(&sm.o_full, (g + T - 1) & 1, abort_flag, st, kSiteOFull, u)) break;
+      // this group's last PV of the unit
+      if (!first) {
+        if (!warp_wait(&sm.o_full[grp], last_use & 1, abort_flag, st, kSiteOFull, u)) break;
         tc_fence_after();
       }
+      if (grp == 1) {
+        sm.mB[s][r] = m;
+        sm.lB[s][r] = l;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm.b_done);
+          mbar_arrive(&sm.route_empty[s]);
+        }
+        g += T;
+        continue;
+      }
+      // ---------------- epilogue (group A): merge A, B and the correction ----------------
+      if (!warp_wait(&sm.b_done, n & 1, abort_flag, st, kSiteBDone, u)) break;
+      const bool hasA = !first;
+      const int tilesB = ((g & 1u) == 1u) ? (T + 1) / 2 : T / 2;
+      const bool hasB = tilesB > 0;
+      const float mB = sm.mB[s][r], lB = sm.lB[s][r];
       const float mc = sm.cmax[s][blk] * kLog2e;
       const float cd = sm.cden[s][blk];
-      const float mf = fmaxf(m, mc);
-      const float a = (m == -INFINITY) ? 0.f : ex2_approx(m - mf);
-      const float c = (mc == -INFINITY) ? 0.f : ex2_approx(mc - mf);
-      const float L = fmaf(l, a, cd * c);
+      const float mf = fmax3(m, mB, mc);
+      const float wa = (m == -INFINITY) ? 0.f : ex2_approx(m - mf);
+      const float wb = (mB == -INFINITY) ? 0.f : ex2_approx(mB - mf);
+      const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - mf);
+      const float L = fmaf(l, wa, fmaf(lB, wb, cd * wc));
       const float inv = 1.f / L;
       const int row = pair * kBM + r;
       const bool valid = row < P.N;
       uint16_t* orow = P.out + (static_cast<long long>(bh) * P.N + row) * D;
+      for (int ch = 0; ch < D / 16; ++ch) {
+        float y[16];
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t ov[32];
-        if (T >= 1) {
-          tmem_ld32(tmem + kColO + ch * 32 + lane_off, ov);
-          tmem_wait_ld();
-        } else {
+        for (int e = 0; e < 16; ++e) y[e] = 0.f;
+        if constexpr (ROUTE) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = 0u;
+          for (int e = 0; e < 16; ++e) y[e] = sm.cnum[s][blk][ch * 16 + e] * wc;
         }
-        uint32_t packed[16];
+        uint32_t o[16];
+        if (hasA) {
+          tmem_ld16(colO + ch * 16, o);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float y0, y1;
-          if constexpr (ROUTE) {
-            const float* cn = &sm.cnum[s][blk][ch * 32 + e];
-            y0 = fmaf(__uint_as_float(ov[e]), a, cn[0] * c) * inv;
-            y1 = fmaf(__uint_as_float(ov[e + 1]), a, cn[1] * c) * inv;
-          } else {
-            y0 = __uint_as_float(ov[e]) * a * inv;
-            y1 = __uint_as_float(ov[e + 1]) * a * inv;
-          }
-          packed[e / 2] = pack_bf16x2(y0, y1);
+          for (int e = 0; e < 16; ++e) y[e] = fmaf(__uint_as_float(o[e]), wa, y[e]);
+        }
+        if (hasB) {
+          tmem_ld16(colO + 128 + ch * 16, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[e] = fmaf(__uint_as_float(o[e]), wb, y[e]);
         }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+          uint32_t pk[8];
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(packed[4 * x], packed[4 * x + 1], packed[4 * x + 2], packed[4 * x + 3]);
+          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(y[2 * e] * inv, y[2 * e + 1] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
       if (valid && P.lse) P.lse[static_cast<long long>(bh) * P.N + row] = (mf + __log2f(L)) * kLn2;
@@ -663,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -734,6 +989,12 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
 }
 
 }  // namespace
+
+#ifdef SOLATTN_TRACE
+extern "C" int solattn_trace_read(unsigned long long* host, size_t n) {
+  return cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 4;
+}
+#endif
 
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   if (a.d == 64) return a.route ? launch_fwd_t<64, true>(a, num_sms, stream) : launch_fwd_t<64, false>(a, num_sms, stream);
