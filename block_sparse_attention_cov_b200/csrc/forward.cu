@@ -479,16 +479,57 @@ __device__ __forceinline__ bool softmax_max(uint32_t (&sv)[32], uint32_t (&sw)[3
   return false;
 }
 
+// 2^y for two packed fp32 values on the FMA pipe (relieves the MUFU unit):
+// Cody-Waite split y = n + f with n = round(y) (adding 1.5 * 2^23 leaves n in
+// the low mantissa bits), f in [-1/2, 1/2], 2^f by the degree-3 minimax
+// polynomial fitted by fit_exp2_poly.py (max relative error 7.5e-5, below
+// the bf16 rounding of P), and n added to the exponent field with one integer
+// multiply-add. y is clamped to >= -125 so 2^n stays a normal float (keys
+// masked to -inf give 2^-125 ~ 2e-38, against a zero V row).
+constexpr float kPolyC0 = 0.9999280571937561f, kPolyC1 = 0.6932609677314758f;
+constexpr float kPolyC2 = 0.2426111400127411f, kPolyC3 = 0.0551716648042202f;
+constexpr int kPolyPairs = 0;  // column pairs per 16-column slice evaluated by the polynomial (0 = all MUFU)
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2_dup(float x) { return f2_from_bits(__float_as_uint(x), __float_as_uint(x)); }
+
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& p0, float& p1) {
+  const uint64_t x = f2_from_bits(__float_as_uint(fmaxf(y0, -125.f)), __float_as_uint(fmaxf(y1, -125.f)));
+  const uint64_t t = fadd2(x, f2_dup(12582912.f));           // 1.5 * 2^23 + round(y)
+  const uint64_t n = fadd2(t, f2_dup(-12582912.f));          // round(y)
+  const uint64_t f = ffma2(n, f2_dup(-1.f), x);              // y - round(y)
+  uint64_t q = ffma2(f2_dup(kPolyC3), f, f2_dup(kPolyC2));
+  q = ffma2(q, f, f2_dup(kPolyC1));
+  q = ffma2(q, f, f2_dup(kPolyC0));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  // exponent += n: the low bits of t hold n, (bits(t) << 23) == n << 23 (mod 2^32)
+  p0 = __int_as_float(static_cast<int>(__float_as_uint(t0) * 8388608u + __float_as_uint(q0)));
+  p1 = __int_as_float(static_cast<int>(__float_as_uint(t1) * 8388608u + __float_as_uint(q1)));
+}
+
 // P for 16 consecutive columns (x holds their raw S bits): 8 packed bf16x2
-// words; adds the fp32 probabilities to l.
+// words; adds the fp32 probabilities to l. The first 8 - kPolyPairs column
+// pairs use the MUFU ex2, the others the FMA-pipe polynomial.
 __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, uint64_t nm2, float& l,
                                               uint32_t (&pw)[8]) {
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int c = 0; c < 16; c += 2) {
-    float y0, y1;
+    float y0, y1, p0, p1;
     f2_split(ffma2(f2_from_bits(x[c], x[c + 1]), sc2, nm2), y0, y1);
-    const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);  // ex2(-inf) = 0 for masked keys
+    if ((c >> 1) < 8 - kPolyPairs) {
+      p0 = ex2_approx(y0);  // ex2(-inf) = 0 for masked keys
+      p1 = ex2_approx(y1);
+    } else {
+      exp2_poly2(y0, y1, p0, p1);
+    }
     if (c & 2) a1 += p0 + p1; else a0 += p0 + p1;
     pw[c >> 1] = pack_bf16x2(p0, p1);
   }
@@ -677,63 +718,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) break;
       }
-      int nq = 0, np = 0;
+      // per softmax group w: next tile to multiply by K (nq[w]) and by V (np[w]);
+      // a group's tiles are t = t0[w], t0[w] + 2, ... (global tile parity)
+      int nq[2], np[2];
+      const int t0 = (g & 1u) ? 1 : 0;  // first unit tile of group 0
+      nq[0] = np[0] = t0;
+      nq[1] = np[1] = 1 - t0;
+      int qk_issued = 0, pv_issued = 0;
       bool ofree_seen = n == 0;
       uint32_t first_pv = 3u;  // bit w: group w has not accumulated into its O in this unit
       unsigned long long t_idle = 0;
-      while (np < T) {
+      while (pv_issued < T) {
         bool progressed = false;
-        if (np < nq) {
-          const uint32_t gp = g + np, stp = gp % kStages, w = gp & 1, usep = gp >> 1;
-          if (!ofree_seen) ofree_seen = __all_sync(0xffffffffu, mbar_test(&sm.o_free, (n - 1) & 1));
-          if (ofree_seen && __all_sync(0xffffffffu, mbar_test(&sm.p_full[w], usep & 1) &&
-                                                         mbar_test(&sm.v_full[stp], (gp / kStages) & 1))) {
-            tc_fence_after();
-            if (elect_one()) {
-              SOLATTN_TRACE_EVENT(11, gp);
-              const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
-              const uint32_t acc0 = (first_pv >> w) & 1u ? 0u : 1u;
 #pragma unroll
-              for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_ts(tmem + kColO + w * 128, tmem + kColP + w * 32 + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
-                       kk > 0 ? 1u : acc0);
-              mma_commit(&sm.v_empty[stp]);
-              mma_commit(&sm.o_full[w]);
+        for (int w = 0; w < 2; ++w) {
+          if (np[w] < nq[w]) {  // PV of group w's oldest multiplied tile
+            const uint32_t gp = g + np[w], stp = gp % kStages, usep = gp >> 1;
+            if (!ofree_seen) ofree_seen = __all_sync(0xffffffffu, mbar_test(&sm.o_free, (n - 1) & 1));
+            if (ofree_seen && __all_sync(0xffffffffu, mbar_test(&sm.p_full[w], usep & 1) &&
+                                                           mbar_test(&sm.v_full[stp], (gp / kStages) & 1))) {
+              tc_fence_after();
+              if (elect_one()) {
+                SOLATTN_TRACE_EVENT(11, gp);
+                const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
+                const uint32_t acc0 = (first_pv >> w) & 1u ? 0u : 1u;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                  mma_ts(tmem + kColO + w * 128, tmem + kColP + w * 32 + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                         kk > 0 ? 1u : acc0);
+                mma_commit(&sm.v_empty[stp]);
+                mma_commit(&sm.o_full[w]);
+              }
+              __syncwarp();
+              first_pv &= ~(1u << w);
+              np[w] += 2;
+              ++pv_issued;
+              progressed = true;
             }
-            __syncwarp();
-            first_pv &= ~(1u << w);
-            ++np;
-            progressed = true;
           }
-        }
-        if (nq < T) {
-          const uint32_t gt = g + nq, stg = gt % kStages, w = gt & 1, use = gt >> 1;
-          if (__all_sync(0xffffffffu, mbar_test(&sm.k_full[stg], (gt / kStages) & 1) &&
-                                          (use == 0 || mbar_test(&sm.s_free[w], (use - 1) & 1)))) {
-            tc_fence_after();
-            if (elect_one()) {
-              const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
+          if (nq[w] < T) {  // QK of group w's next tile
+            const uint32_t gt = g + nq[w], stg = gt % kStages, use = gt >> 1;
+            if (__all_sync(0xffffffffu, mbar_test(&sm.k_full[stg], (gt / kStages) & 1) &&
+                                            (use == 0 || mbar_test(&sm.s_free[w], (use - 1) & 1)))) {
+              tc_fence_after();
+              if (elect_one()) {
+                const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk)
-                mma_ts(tmem + kColS + w * 64, tmem + kColQ + kk * 8,
-                       kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
-              mma_commit(&sm.s_full[w]);
-              mma_commit(&sm.k_empty[stg]);
-              if (nq == T - 1) mma_commit(&sm.q_free);
-              SOLATTN_TRACE_EVENT(10, gt);
+                for (int kk = 0; kk < D / 16; ++kk)
+                  mma_ts(tmem + kColS + w * 64, tmem + kColQ + kk * 8,
+                         kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+                mma_commit(&sm.s_full[w]);
+                mma_commit(&sm.k_empty[stg]);
+                if (qk_issued == T - 1) mma_commit(&sm.q_free);
+                SOLATTN_TRACE_EVENT(10, gt);
+              }
+              __syncwarp();
+              nq[w] += 2;
+              ++qk_issued;
+              progressed = true;
             }
-            __syncwarp();
-            ++nq;
-            progressed = true;
           }
         }
         if (progressed) {
           t_idle = 0;
-        } else {  // bounded: give up if nothing became ready for the wait budget
+        } else {
+          // nothing ready: sleep briefly on the most likely next event (a P
+          // buffer), so the spin does not take issue slots from softmax warps
+          const int w = (np[0] < nq[0]) ? 0 : 1;
+          const uint32_t gp = g + np[w];
+          mbar_try_wait_ns(&sm.p_full[w], (gp >> 1) & 1, 200);
           const unsigned long long now = global_timer_ns();
           if (t_idle == 0) {
             t_idle = now;
-          } else if (now - t_idle > kWaitBudgetNs || *abort_flag) {
+          } else if (now - t_idle > kWaitBudgetNs || *abort_flag) {  // bounded
             if (lane == 0 && !*abort_flag && atomicCAS(&st->error, 0u, kErrTimeout) == 0u) {
               st->where = kSiteMmaStall;
               st->unit = static_cast<uint32_t>(u);
@@ -796,14 +853,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm.s_free[grp]);
         float rescale = 1.f;
         bool need = false;
-        if (mine) need = softmax_max(sv, sw, (j == P.NB - 1) ? nlast : kBN, sl2, m, rescale);
-        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 2, gt);
-        // this group's previous PV must be complete: it read P and wrote O
+        uint32_t pw[32];
+        if (mine) {
+          need = softmax_max(sv, sw, (j == P.NB - 1) ? nlast : kBN, sl2, m, rescale);
+          if (need) l *= rescale;
+          if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 2, gt);
+          const uint64_t sc2 = f2_dup(sl2);
+          const uint64_t nm2 = f2_dup(-m);
+          softmax_slice(&sv[0], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[0]));
+          softmax_slice(&sv[16], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[8]));
+          softmax_slice(&sw[0], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[16]));
+          softmax_slice(&sw[16], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[24]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pw[c] = 0u;
+        }
+        // this group's previous PV must be complete: it read the P buffer and wrote O
         if (!first && !warp_wait(&sm.o_full[grp], (use - 1) & 1, abort_flag, st, kSiteOFull, u)) { ok = false; break; }
         tc_fence_after();
         if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 3, gt);
         if (__any_sync(0xffffffffu, need)) {
-          l *= rescale;
 #pragma unroll
           for (int ch = 0; ch < D / 16; ++ch) {
             uint32_t ov[16];
@@ -814,25 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(colO + ch * 16, ov);
           }
         }
-        if (mine) {
-          const uint64_t sc2 = f2_from_bits(__float_as_uint(sl2), __float_as_uint(sl2));
-          const uint64_t nm2 = f2_from_bits(__float_as_uint(-m), __float_as_uint(-m));
-          uint32_t pw[8];
-          softmax_slice(&sv[0], sc2, nm2, l, pw);
-          tmem_st8(colP, pw);
-          softmax_slice(&sv[16], sc2, nm2, l, pw);
-          tmem_st8(colP + 8, pw);
-          softmax_slice(&sw[0], sc2, nm2, l, pw);
-          tmem_st8(colP + 16, pw);
-          softmax_slice(&sw[16], sc2, nm2, l, pw);
-          tmem_st8(colP + 24, pw);
-        } else {
-          uint32_t z[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) z[c] = 0u;
-          tmem_st16(colP, z);
-          tmem_st16(colP + 16, z);
-        }
+        tmem_st32(colP, pw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
