@@ -15,6 +15,7 @@ EXPORTS = (
     "solattn_status",
     "solattn_strerror",
     "solattn_version",
+    "solattn_forward_noalloc",
 )
 
 OK = 0
@@ -25,7 +26,9 @@ ERR_CUDA = 4
 ERR_TIMEOUT = 5
 ERR_DEVICE = 6
 ERR_WORKSPACE = 7
+ERR_SCRATCH = 8
 WORKSPACE_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 16 << 20
 BLOCK = 64
 MAX_TOKENS = 262144
 
@@ -62,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.solattn_status.restype = i
     L.solattn_strerror.argtypes = [i]
     L.solattn_strerror.restype = ctypes.c_char_p
+    L.solattn_forward_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
+    L.solattn_forward_noalloc.restype = i
     L.solattn_version.argtypes = []
     L.solattn_version.restype = i
     _lib = L

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/solattn.h"
 #include "kernels.h"
@@ -126,6 +127,7 @@ const char* solattn_strerror(int code) {
     case SOLATTN_ERR_TIMEOUT: return "a bounded wait inside the kernel expired; outputs are invalid";
     case SOLATTN_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
     case SOLATTN_ERR_WORKSPACE: return "workspace missing or smaller than SOLATTN_WORKSPACE_BYTES";
+    case SOLATTN_ERR_SCRATCH: return "problem too large for the static scratch of solattn_forward_noalloc";
     default: return "unknown status code";
   }
 }
@@ -195,6 +197,61 @@ int solattn_status(const void* workspace, void* stream) {
   DeviceStatus h{};
   if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SOLATTN_ERR_CUDA;
   return h.error == 0 ? SOLATTN_OK : static_cast<int>(h.error);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: pooled statistics and workspace live in a static
+// device array instead of caller-provided buffers.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SOLATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Device address of the static scratch on the current device (looked up once
+// per device, with that device current), or nullptr on failure.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int solattn_forward_noalloc(const void* q, const void* k, const void* v, int B, int H, int N, int d, float beta,
+                            void* out, float* lse, int32_t* density_out, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_qkv(q, k, v))) return rc;
+  if (!out) return SOLATTN_ERR_ARG;
+  if (!aligned16(out)) return SOLATTN_ERR_ALIGN;
+  if ((lse && !aligned4(lse)) || (density_out && !aligned4(density_out))) return SOLATTN_ERR_ALIGN;
+  if (std::isnan(beta)) return SOLATTN_ERR_ARG;
+  size_t pooled_bytes = 0;
+  if ((rc = solattn_pooled_layout(B, H, N, d, nullptr, nullptr, &pooled_bytes))) return rc;
+  const size_t need = SOLATTN_WORKSPACE_BYTES + pooled_bytes;
+  if (need > SOLATTN_NOALLOC_SCRATCH_BYTES) return SOLATTN_ERR_SCRATCH;
+  int sms = 0;
+  if ((rc = current_device_sms(&sms))) return rc;
+  char* scratch = static_cast<char*>(noalloc_scratch_address());
+  if (!scratch) return SOLATTN_ERR_CUDA;
+  solattn_pooled_t pooled;
+  if ((rc = solattn_pooled_layout(B, H, N, d, scratch + SOLATTN_WORKSPACE_BYTES, &pooled, nullptr))) return rc;
+  if ((rc = solattn_pool(q, k, v, B, H, N, d, &pooled, stream))) return rc;
+  return solattn_forward(q, k, v, B, H, N, d, &pooled, beta, out, lse, density_out, scratch,
+                         SOLATTN_WORKSPACE_BYTES, stream);
 }
 
 }  // extern "C"

@@ -53,7 +53,8 @@ enum solattn_status_code {
   SOLATTN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
   SOLATTN_ERR_TIMEOUT = 5,     /* a bounded device wait expired (device side) */
   SOLATTN_ERR_DEVICE = 6,      /* current device is not an sm_100 GPU */
-  SOLATTN_ERR_WORKSPACE = 7    /* workspace missing or smaller than SOLATTN_WORKSPACE_BYTES */
+  SOLATTN_ERR_WORKSPACE = 7,   /* workspace missing or smaller than SOLATTN_WORKSPACE_BYTES */
+  SOLATTN_ERR_SCRATCH = 8      /* problem needs more than SOLATTN_NOALLOC_SCRATCH_BYTES of scratch */
 };
 
 /*
@@ -143,6 +144,34 @@ int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int
  * synchronisation or the read fails.
  */
 int solattn_status(const void* workspace, void* stream);
+
+/*
+ * Allocation-free forward, for callers that cannot allocate device memory
+ * themselves: code running where cudaMalloc is unavailable or forbidden (for
+ * example inside a host framework that owns every allocation, a plugin that
+ * may only receive tensors, or an embedded runtime with a fixed memory plan).
+ * There is no counterpart on the pages: it is solattn_pool followed by
+ * solattn_forward, with the pooled statistics and the workspace placed in one
+ * file-scope static device array of SOLATTN_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading this library holds until the process exits.
+ *
+ * Arguments, layouts and results are those of solattn_pool + solattn_forward
+ * (the caller passes inputs and outputs only; lse and density_out may be NULL).
+ * The scratch needed is SOLATTN_WORKSPACE_BYTES plus the solattn_pooled_layout
+ * size; larger problems are rejected with SOLATTN_ERR_SCRATCH before anything is
+ * enqueued. Nothing is allocated (no cudaMalloc, cudaFree or allocating library
+ * call). The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. All calls share the one array and it keeps the last
+ * call's contents: calls that overlap on the GPU (other streams, other host
+ * threads) race and must be serialised by the caller. The scheduler counter and
+ * status word at the start of the array are cleared by every call; the status
+ * word is not exposed (a bounded device wait that expires still ends the kernel
+ * early instead of hanging, but this call cannot report it).
+ */
+#define SOLATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+int solattn_forward_noalloc(const void* q, const void* k, const void* v, int B, int H, int N, int d, float beta,
+                            void* out, float* lse, int32_t* density_out, void* stream);
 
 /* Static description of a status code. */
 const char* solattn_strerror(int code);

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_version_and_strerror(L):
     assert L.solattn_version() == 10000
-    for code in range(0, 8):
+    for code in range(0, 9):
         assert _lib.strerror(code) and "unknown" not in _lib.strerror(code)
     assert "unknown" in _lib.strerror(99)
 
