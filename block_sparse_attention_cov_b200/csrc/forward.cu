@@ -41,7 +41,7 @@ namespace solattn {
 
 #ifdef SOLATTN_TRACE
 // Debug builds only: per-tile timestamps of CTA 0 (clock64), [event][index].
-__device__ unsigned long long g_trace[16][4096];
+__device__ unsigned long long g_trace[40][4096];
 #define SOLATTN_TRACE_EVENT(ev, idx)                                         \
   do {                                                                       \
     if (blockIdx.x == 0 && (idx) < 4096) g_trace[(ev)][(idx)] = clock64();   \
@@ -115,7 +115,7 @@ struct __align__(1024) Smem {
   uint64_t o_free, b_done, q_free;
   uint64_t route_full[2], route_empty[2];
   uint64_t rfull[2];                 // routing chunk buffers landed
-  uint64_t mma_done;
+  uint64_t mma_done[2];
   float mB[2][kBM];                  // group B's final running max / sum per row, per slot
   float lB[2][kBM];
   uint32_t tmem_base;
@@ -543,9 +543,8 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
 //   warps 8-11  routing, one unit ahead (Q rows into TMEM after the previous
 //               unit's last QK has completed)
 //   warp 12     TMA producer of the K tiles of the kept list
-//   warp 13     MMA issuer (event loop, one elected lane issues)
+//   warps 13/15 MMA issuers of group A / group B (one elected lane issues)
 //   warp 14     TMA producer of the V tiles
-//   warp 15     idle (completes the last warpgroup for register rebalancing)
 // TMEM: Q at 0 (64 columns), S_A/S_B at 64/128, P_A/P_B at 192/224,
 // O_A/O_B at 256/384. Each group keeps its own running max, sum and O; the
 // epilogue merges the two with the skipped-block correction.
@@ -574,13 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[i], 4);
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.route_full[i], 1);
-      mbar_init(&sm.route_empty[i], 11);  // 2 producers + MMA + 8 softmax warps
+      mbar_init(&sm.route_empty[i], 12);  // 2 producers + 2 MMA issuers + 8 softmax warps
       mbar_init(&sm.rfull[i], 1);
     }
     mbar_init(&sm.o_free, 4);
     mbar_init(&sm.b_done, 4);
-    mbar_init(&sm.q_free, 1);
-    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.q_free, 2);  // one commit per MMA issuer
+    mbar_init(&sm.mma_done[0], 1);
+    mbar_init(&sm.mma_done[1], 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -692,20 +692,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t gt = first; gt < g; ++gt) mbar_wait_quiet(&full[gt % kStages], (gt / kStages) & 1);
     }
     __syncwarp();
-  } else if (warp == 15) {
-    // idle warp (completes the last warpgroup)
-  } else if (warp == 13) {
-    // ======================= MMA issuer =======================
-    // Event loop: issues QK of the next tile whose K tile has landed and whose
-    // S buffer its group has read, and PV of the next tile whose P is ready,
-    // whichever is ready first (QKs in tile order, PVs in tile order).
+  } else if (warp == 13 || warp == 15) {
+    // ======================= MMA issuers: warp 13 for group A, warp 15 for group B =======================
+    // For the group's own tiles t (global tile parity = group): QK of the next
+    // own tile as soon as the group has read the S of the current one (one S
+    // buffer per group), then PV of the current one once its P is stored.
+    // Waits sleep on their mbarrier (bounded); one lane issues.
+    const int grp = warp == 13 ? 0 : 1;
     constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
     constexpr uint32_t kTileBytes = kBN * D * 2;
     const uint64_t kdesc0 = sw128_desc(smem_u32(&sm.kt[0][0]), 16, 1024);
     const uint64_t vdesc0 = sw128_desc(smem_u32(&sm.vt[0][0]), 8192, 1024);
+    const uint32_t colS = tmem + kColS + grp * 64, colP = tmem + kColP + grp * 32, colO = tmem + kColO + grp * 128;
     uint32_t g = 0;
     bool ok = true;
+    auto issue_qk = [&](uint32_t gt, int u, bool last) -> bool {
+      const uint32_t stg = gt % kStages, use = gt >> 1;
+      if (use >= 1 && !warp_wait(&sm.s_free[grp], (use - 1) & 1, abort_flag, st, kSiteSFree, u)) return false;
+      if (!warp_wait(&sm.k_full[stg], (gt / kStages) & 1, abort_flag, st, kSiteKFull, u)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(colS, tmem + kColQ + kk * 8, kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&sm.s_full[grp]);
+        mma_commit(&sm.k_empty[stg]);
+        if (last) mma_commit(&sm.q_free);
+        SOLATTN_TRACE_EVENT(10, gt);
+      }
+      __syncwarp();
+      return true;
+    };
     for (int n = 0; ok; ++n) {
       const int s = n & 1;
       if (!warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullMma, 0)) break;
@@ -713,92 +733,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      if (T == 0) {
+      const int t0 = ((g & 1u) == static_cast<uint32_t>(grp)) ? 0 : 1;  // first own tile of the unit
+      if (t0 >= T) {  // no own tile: still release the Q slot and keep o_free's phase
         if (elect_one()) mma_commit(&sm.q_free);
         __syncwarp();
         if (n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) break;
-      }
-      // per softmax group w: next tile to multiply by K (nq[w]) and by V (np[w]);
-      // a group's tiles are t = t0[w], t0[w] + 2, ... (global tile parity)
-      int nq[2], np[2];
-      const int t0 = (g & 1u) ? 1 : 0;  // first unit tile of group 0
-      nq[0] = np[0] = t0;
-      nq[1] = np[1] = 1 - t0;
-      int qk_issued = 0, pv_issued = 0;
-      bool ofree_seen = n == 0;
-      uint32_t first_pv = 3u;  // bit w: group w has not accumulated into its O in this unit
-      unsigned long long t_idle = 0;
-      while (pv_issued < T) {
-        bool progressed = false;
+      } else {
+        ok = issue_qk(g + t0, u, t0 + 2 >= T);
+        if (ok && n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) ok = false;
+        for (int t = t0; t < T && ok; t += 2) {
+          if (t + 2 < T && !(ok = issue_qk(g + t + 2, u, t + 4 >= T))) break;
+          const uint32_t gp = g + t, stp = gp % kStages, usep = gp >> 1;
+          if (!warp_wait(&sm.p_full[grp], usep & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
+          if (!warp_wait(&sm.v_full[stp], (gp / kStages) & 1, abort_flag, st, kSiteVFull, u)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
+            SOLATTN_TRACE_EVENT(11, gp);
+            const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (np[w] < nq[w]) {  // PV of group w's oldest multiplied tile
-            const uint32_t gp = g + np[w], stp = gp % kStages, usep = gp >> 1;
-            if (!ofree_seen) ofree_seen = __all_sync(0xffffffffu, mbar_test(&sm.o_free, (n - 1) & 1));
-            if (ofree_seen && __all_sync(0xffffffffu, mbar_test(&sm.p_full[w], usep & 1) &&
-                                                           mbar_test(&sm.v_full[stp], (gp / kStages) & 1))) {
-              tc_fence_after();
-              if (elect_one()) {
-                SOLATTN_TRACE_EVENT(11, gp);
-                const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
-                const uint32_t acc0 = (first_pv >> w) & 1u ? 0u : 1u;
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                  mma_ts(tmem + kColO + w * 128, tmem + kColP + w * 32 + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
-                         kk > 0 ? 1u : acc0);
-                mma_commit(&sm.v_empty[stp]);
-                mma_commit(&sm.o_full[w]);
-              }
-              __syncwarp();
-              first_pv &= ~(1u << w);
-              np[w] += 2;
-              ++pv_issued;
-              progressed = true;
-            }
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ts(colO, colP + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (t > t0 || kk > 0) ? 1u : 0u);
+            mma_commit(&sm.v_empty[stp]);
+            mma_commit(&sm.o_full[grp]);
           }
-          if (nq[w] < T) {  // QK of group w's next tile
-            const uint32_t gt = g + nq[w], stg = gt % kStages, use = gt >> 1;
-            if (__all_sync(0xffffffffu, mbar_test(&sm.k_full[stg], (gt / kStages) & 1) &&
-                                            (use == 0 || mbar_test(&sm.s_free[w], (use - 1) & 1)))) {
-              tc_fence_after();
-              if (elect_one()) {
-                const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                  mma_ts(tmem + kColS + w * 64, tmem + kColQ + kk * 8,
-                         kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
-                mma_commit(&sm.s_full[w]);
-                mma_commit(&sm.k_empty[stg]);
-                if (qk_issued == T - 1) mma_commit(&sm.q_free);
-                SOLATTN_TRACE_EVENT(10, gt);
-              }
-              __syncwarp();
-              nq[w] += 2;
-              ++qk_issued;
-              progressed = true;
-            }
-          }
-        }
-        if (progressed) {
-          t_idle = 0;
-        } else {
-          // nothing ready: sleep briefly on the most likely next event (a P
-          // buffer), so the spin does not take issue slots from softmax warps
-          const int w = (np[0] < nq[0]) ? 0 : 1;
-          const uint32_t gp = g + np[w];
-          mbar_try_wait_ns(&sm.p_full[w], (gp >> 1) & 1, 200);
-          const unsigned long long now = global_timer_ns();
-          if (t_idle == 0) {
-            t_idle = now;
-          } else if (now - t_idle > kWaitBudgetNs || *abort_flag) {  // bounded
-            if (lane == 0 && !*abort_flag && atomicCAS(&st->error, 0u, kErrTimeout) == 0u) {
-              st->where = kSiteMmaStall;
-              st->unit = static_cast<uint32_t>(u);
-            }
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
+          __syncwarp();
         }
       }
       if (!ok) break;
@@ -806,9 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       g += T;
     }
-    if (elect_one()) mma_commit(&sm.mma_done);  // teardown: issued MMAs complete before TMEM is freed
+    if (elect_one()) mma_commit(&sm.mma_done[grp]);  // teardown: issued MMAs complete before TMEM is freed
     __syncwarp();
-    mbar_wait_quiet(&sm.mma_done, 0);
+    mbar_wait_quiet(&sm.mma_done[grp], 0);
     __syncwarp();
   } else {
     // ======================= softmax groups A (warps 0-3) and B (4-7) =======================

@@ -11,9 +11,9 @@
 //   pool_means_kernel  -- HBM-bound: reads q, k, v once with 128-bit loads and
 //                         writes the fp32 block means (qbar, kbar, vbar).
 //   key_stats_kernel   -- per head: mean of kbar and its covariance (two-pass,
-//                         divided by N_b), one 64x64 tile of it per CTA.
+//                         divided by N_b), one 32x32 tile (and its mirror) per CTA.
 //   row_stats_kernel   -- per query block: mu_i = s qbar_i . kmean and
-//                         sigma_i = s sqrt(max(0, qbar_i^T C qbar_i)).
+//                         sigma_i = s sqrt(max(0, qbar_i^T C qbar_i)), 64 blocks per CTA.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -102,126 +102,149 @@ __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restr
   }
 }
 
-// grid = (T*T, BH) with T = D/64; CTA (ta, tb) writes kcov[ta*64.., tb*64..].
+// Covariance of the pooled keys, two-pass. grid = (number of 32x32 tiles on or
+// above the diagonal, BH); CTA (ta <= tb) computes tile (ta, tb) and writes it
+// and its mirror (tb, ta). Pass 1: mean of the 64 columns it needs (fixed
+// order); pass 2: sum over key blocks of the deviations' outer products, 64
+// key blocks staged in shared memory per trip.
 template <int D>
 __global__ void __launch_bounds__(256) key_stats_kernel(const float* __restrict__ kbar, float* __restrict__ kmean,
                                                         float* __restrict__ kcov, int NB) {
-  constexpr int T = D / 64;
-  constexpr int JC = 32;  // pooled keys staged per trip
-  __shared__ float mean_part[256 / D][D];
-  __shared__ float mean_s[D];
-  __shared__ float da[JC][64];
-  __shared__ float db[JC][64];
+  constexpr int T = D / 32;
+  constexpr int JC = 128;
+  __shared__ float mpart[8][64];
+  __shared__ float mcol[64];        // means of columns ta*32.. (0-31) and tb*32.. (32-63)
+  __shared__ float da[JC][33];      // deviations, padded against bank conflicts
+  __shared__ __align__(16) float db[JC][32];
   const int tid = threadIdx.x;
   const int bh = blockIdx.y;
-  const int ta = blockIdx.x / T, tb = blockIdx.x % T;
+  int ta = 0, tb = 0;
+  {  // blockIdx.x -> (ta, tb), ta <= tb, row-major over the upper triangle
+    int rem = blockIdx.x;
+    for (ta = 0; ta < T; ++ta) {
+      if (rem < T - ta) { tb = ta + rem; break; }
+      rem -= T - ta;
+    }
+  }
   const float* kb = kbar + static_cast<long long>(bh) * NB * D;
-  // pass 1: mean, fixed summation order
   {
-    const int col = tid % D, part = tid / D;
-    float s = 0.f;
-    for (int j = part; j < NB; j += 256 / D) s += kb[static_cast<long long>(j) * D + col];
-    mean_part[part][col] = s;
+    // 4 partial sums per column, each over rows part, part + 4, ...; 8
+    // independent accumulators keep 8 loads in flight (fixed summation order)
+    const int c = tid % 64, part = tid / 64;
+    const int col = c < 32 ? ta * 32 + c : tb * 32 + (c - 32);
+    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int j = part;
+    for (; j + 28 < NB; j += 32) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc8[u] += kb[static_cast<long long>(j + 4 * u) * D + col];
+    }
+    for (int u = 0; j < NB; j += 4, ++u) acc8[u & 7] += kb[static_cast<long long>(j) * D + col];
+    mpart[part][c] = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
   }
   __syncthreads();
-  if (tid < D) {
-    float s = 0.f;
-#pragma unroll
-    for (int p = 0; p < 256 / D; ++p) s += mean_part[p][tid];
-    mean_s[tid] = s / static_cast<float>(NB);
-    if (blockIdx.x == 0) kmean[static_cast<long long>(bh) * D + tid] = mean_s[tid];
+  if (tid < 64) {
+    mcol[tid] = ((mpart[0][tid] + mpart[1][tid]) + (mpart[2][tid] + mpart[3][tid])) / static_cast<float>(NB);
+    if (ta == tb && tid < 32) kmean[static_cast<long long>(bh) * D + ta * 32 + tid] = mcol[tid];
   }
   __syncthreads();
-  // pass 2: covariance tile from deviations
-  const int a0 = (tid / 16) * 4, b0 = (tid % 16) * 4;
-  float acc[4][4];
-#pragma unroll
-  for (int x = 0; x < 4; ++x)
-#pragma unroll
-    for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+  const int a = tid / 8, b0 = (tid % 8) * 4;  // this thread: row a, columns b0..b0+3 of the tile
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int j0 = 0; j0 < NB; j0 += JC) {
-    for (int e = tid; e < JC * 64; e += 256) {
-      const int jj = e / 64, cc = e % 64, j = j0 + jj;
+    for (int e = tid; e < JC * 32; e += 256) {
+      const int jj = e / 32, cc = e % 32, j = j0 + jj;
       const bool ok = j < NB;
-      da[jj][cc] = ok ? kb[static_cast<long long>(j) * D + ta * 64 + cc] - mean_s[ta * 64 + cc] : 0.f;
-      db[jj][cc] = ok ? kb[static_cast<long long>(j) * D + tb * 64 + cc] - mean_s[tb * 64 + cc] : 0.f;
+      da[jj][cc] = ok ? kb[static_cast<long long>(j) * D + ta * 32 + cc] - mcol[cc] : 0.f;
+      db[jj][cc] = ok ? kb[static_cast<long long>(j) * D + tb * 32 + cc] - mcol[32 + cc] : 0.f;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
     for (int jj = 0; jj < JC; ++jj) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) av[x] = da[jj][a0 + x];
-#pragma unroll
-      for (int y = 0; y < 4; ++y) bv[y] = db[jj][b0 + y];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+      const float x = da[jj][a];
+      const float4 y = *reinterpret_cast<const float4*>(&db[jj][b0]);
+      acc[0] = fmaf(x, y.x, acc[0]);
+      acc[1] = fmaf(x, y.y, acc[1]);
+      acc[2] = fmaf(x, y.z, acc[2]);
+      acc[3] = fmaf(x, y.w, acc[3]);
     }
     __syncthreads();
   }
   const float inv = 1.f / static_cast<float>(NB);
   float* out = kcov + static_cast<long long>(bh) * D * D;
+  const int row = ta * 32 + a, col = tb * 32 + b0;
+  *reinterpret_cast<float4*>(out + static_cast<long long>(row) * D + col) =
+      make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  if (ta != tb) {
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    float4 r = make_float4(acc[x][0] * inv, acc[x][1] * inv, acc[x][2] * inv, acc[x][3] * inv);
-    *reinterpret_cast<float4*>(out + static_cast<long long>(ta * 64 + a0 + x) * D + tb * 64 + b0) = r;
+    for (int x = 0; x < 4; ++x) out[static_cast<long long>(col + x) * D + row] = acc[x] * inv;
   }
 }
 
-// grid = (chunks, BH), 256 threads = 8 warps; dynamic smem holds C (D*D fp32).
+// mu_i = s qbar_i . kmean and sigma_i = s sqrt(max(0, qbar_i^T C qbar_i)) for 64
+// query blocks per CTA: thread t owns block t / 4 and a quarter of the columns
+// of y = C qbar (C symmetric), then reduces qbar . y over the 4 threads.
+// grid = (ceil(NB / 64), BH); dynamic smem = C (D*D) + 64 padded qbar rows.
 template <int D>
 __global__ void __launch_bounds__(256) row_stats_kernel(const float* __restrict__ qbar,
                                                         const float* __restrict__ kmean,
                                                         const float* __restrict__ kcov, float* __restrict__ mu,
                                                         float* __restrict__ sigma, int NB) {
+  constexpr int QS = D + 4;     // padded row stride of the staged qbar rows
+  constexpr int CW = D / 4;     // columns per thread
   extern __shared__ __align__(16) float smem_f[];
   float* C = smem_f;            // [D][D]
-  float* km = C + D * D;        // [D]
-  float* qs = km + D;           // [8][D]
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  float* Q = C + D * D;         // [64][QS]
+  float* km = Q + 64 * QS;      // [D]
+  const int tid = threadIdx.x;
   const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * 64;
   const float* cg = kcov + static_cast<long long>(bh) * D * D;
   for (int e = tid; e < D * D / 4; e += 256)
     reinterpret_cast<float4*>(C)[e] = reinterpret_cast<const float4*>(cg)[e];
+  for (int e = tid; e < 64 * D; e += 256) {
+    const int r = e / D, c = e % D;
+    Q[r * QS + c] = (i0 + r < NB) ? qbar[(static_cast<long long>(bh) * NB + i0 + r) * D + c] : 0.f;
+  }
   if (tid < D) km[tid] = kmean[static_cast<long long>(bh) * D + tid];
   __syncthreads();
-  const float s = rsqrtf(static_cast<float>(D));
-  constexpr int M = D / 32;
-  for (int i = blockIdx.x * 8 + warp; i < NB; i += gridDim.x * 8) {
-    const float* qg = qbar + (static_cast<long long>(bh) * NB + i) * D;
-    float qv[M];
+  // thread (r, c4): columns c4 * 4 + 16 m .. + 3 (m < D / 16): the four threads
+  // of a row read 64 contiguous bytes of C per step (no bank conflicts)
+  const int r = tid / 4, c4 = tid % 4;
+  const float* qrow = Q + r * QS;
+  float y[CW];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      qv[m] = qg[lane + 32 * m];
-      qs[warp * D + lane + 32 * m] = qv[m];
-    }
-    __syncwarp();
-    float y[M];
+  for (int c = 0; c < CW; ++c) y[c] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < D; ++k) {
+    const float qk = qrow[k];
+    const float* crow = C + k * D + c4 * 4;
 #pragma unroll
-    for (int m = 0; m < M; ++m) y[m] = 0.f;
-    for (int b = 0; b < D; ++b) {
-      const float qb = qs[warp * D + b];
+    for (int m = 0; m < CW / 4; ++m) {
+      const float4 cv = *reinterpret_cast<const float4*>(crow + 16 * m);
+      y[4 * m] = fmaf(qk, cv.x, y[4 * m]);
+      y[4 * m + 1] = fmaf(qk, cv.y, y[4 * m + 1]);
+      y[4 * m + 2] = fmaf(qk, cv.z, y[4 * m + 2]);
+      y[4 * m + 3] = fmaf(qk, cv.w, y[4 * m + 3]);
+    }
+  }
+  float quad = 0.f, dot = 0.f;
 #pragma unroll
-      for (int m = 0; m < M; ++m) y[m] = fmaf(C[b * D + lane + 32 * m], qb, y[m]);  // C symmetric
-    }
-    float quad = 0.f, dot = 0.f;
+  for (int m = 0; m < CW / 4; ++m) {
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      quad = fmaf(qv[m], y[m], quad);
-      dot = fmaf(qv[m], km[lane + 32 * m], dot);
+    for (int e = 0; e < 4; ++e) {
+      const int c = c4 * 4 + 16 * m + e;
+      quad = fmaf(qrow[c], y[4 * m + e], quad);
+      dot = fmaf(qrow[c], km[c], dot);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      quad += __shfl_xor_sync(0xffffffffu, quad, off);
-      dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    }
-    if (lane == 0) {
-      mu[static_cast<long long>(bh) * NB + i] = s * dot;
-      sigma[static_cast<long long>(bh) * NB + i] = s * sqrtf(fmaxf(quad, 0.f));
-    }
-    __syncwarp();
+  }
+  quad += __shfl_xor_sync(0xffffffffu, quad, 1);
+  dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+  quad += __shfl_xor_sync(0xffffffffu, quad, 2);
+  dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+  const int i = i0 + r;
+  if ((tid % 4) == 0 && i < NB) {
+    const float s = rsqrtf(static_cast<float>(D));
+    mu[static_cast<long long>(bh) * NB + i] = s * dot;
+    sigma[static_cast<long long>(bh) * NB + i] = s * sqrtf(fmaxf(quad, 0.f));
   }
 }
 
@@ -234,16 +257,15 @@ cudaError_t launch_pool_d(const uint16_t* q, const uint16_t* k, const uint16_t* 
   pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, BH, N, NB);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  constexpr int T = D / 64;
-  key_stats_kernel<D><<<dim3(T * T, BH), 256, 0, stream>>>(p.kbar, p.kmean, p.kcov, NB);
+  constexpr int T = D / 32;
+  key_stats_kernel<D><<<dim3(T * (T + 1) / 2, BH), 256, 0, stream>>>(p.kbar, p.kmean, p.kcov, NB);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = (static_cast<size_t>(D) * D + D + 8 * D) * sizeof(float);
+  const size_t smem = (static_cast<size_t>(D) * D + 64 * (D + 4) + D) * sizeof(float);
   e = cudaFuncSetAttribute(row_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int chunks = (NB + 63) / 64;  // 64 query blocks per CTA
-  row_stats_kernel<D><<<dim3(chunks, BH), 256, smem, stream>>>(p.qbar, p.kmean, p.kcov, p.mu, p.sigma, NB);
+  row_stats_kernel<D><<<dim3((NB + 63) / 64, BH), 256, smem, stream>>>(p.qbar, p.kmean, p.kcov, p.mu, p.sigma, NB);
   return cudaGetLastError();
 }
 
