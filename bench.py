@@ -175,6 +175,21 @@ def oracle_sample(q, k, v, beta, heads, blocks_per_head, seed=0):
     return t_total, flops, desc
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings (ms) over all ranks; identity for
+    one rank. Every rank must call it with the same number of values."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(flops_per_rank, ms, world):
+    """Whole-job throughput in TFLOP/s: every rank processes its own copy of the
+    workload (weak scaling), the job takes the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -269,10 +284,7 @@ def run_ours(args, rank, world, local_rank):
     ms_total = t_start.elapsed_time(t_end)
     pool_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     fwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    ms = torch.tensor([ms_total, pool_ms, fwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-    ms_total, pool_ms, fwd_ms = (float(x) for x in ms.tolist())
+    ms_total, pool_ms, fwd_ms = max_over_ranks([ms_total, pool_ms, fwd_ms], world, dev)
     ms_step = ms_total / args.steps
 
     # dense comparison path on the same inputs
@@ -322,13 +334,11 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = torch.tensor([e0.elapsed_time(e1) / reps], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+        (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp))
         d2h = sum(x.numel() * x.element_size() for x in (out_h, lse_h, dens_h))
-        e2e = {"value": world * kflops / (float(e2e_ms.item()) * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(e2e_ms.item())}
+        e2e = {"value": job_value(kflops, e2e_ms, world), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if rank != 0:
         return
@@ -343,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
                "sample": desc + f"; {secs:.1f} s of CPU time"}
     line = {
         "metric": METRIC,
-        "value": world * kflops / (ms_step * 1e-3) / 1e12,
+        "value": job_value(kflops, ms_step, world),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
