@@ -4,7 +4,7 @@
                     [--workload wan_75k] [--beta B]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-solattn_pool (block means, key covariance, mu/sigma) followed by
+solattn_pool (block means, key mean and covariance) followed by
 solattn_forward (on-the-fly routing, exact kept blocks, zeroth-order correction)
 at the Wan2.1-14B-like 720p shape: 75,600 tokens (21x45x80 latent grid), 40
 heads, d = 128, beta calibrated for a 15 % mean kept-block density.
@@ -125,9 +125,12 @@ def kept_flops(stats, dens, beta, N, d):
     n_i[-1] = n_last
     cols = 64.0 * dens.double()
     if n_last < 64:
-        qbar, kbar = stats.view("qbar"), stats.view("kbar")
-        sh = (qbar.double() @ kbar[..., -1, :].double().unsqueeze(-1)).squeeze(-1) / math.sqrt(d)
-        tau = stats.view("mu").double() + beta * stats.view("sigma").double()
+        qbar, kbar = stats.view("qbar").double(), stats.view("kbar").double()
+        s = 1.0 / math.sqrt(d)
+        sh = s * (qbar @ kbar[..., -1, :].unsqueeze(-1)).squeeze(-1)
+        mu = s * (qbar @ stats.view("kmean").double().unsqueeze(-1)).squeeze(-1)
+        sigma = s * ((qbar @ stats.view("kcov").double()) * qbar).sum(-1).clamp_min(0.0).sqrt()
+        tau = torch.where(sigma == 0, torch.full_like(mu, math.inf), mu + beta * sigma)
         cols = cols - (64 - n_last) * (sh > tau).double()
     return float((4.0 * d * n_i * cols).sum().item())
 
@@ -138,7 +141,7 @@ def dense_flops(B, H, N, d):
 
 def pool_bytes(B, H, N, d):
     nb = math.ceil(N / 64)
-    return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d + 2 * nb) * B * H * 4
+    return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d) * B * H * 4
 
 
 def cpu_threads():

@@ -76,7 +76,7 @@ class PooledStats:
         nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
         dims = {
             "qbar": (B, H, nb, d), "kbar": (B, H, nb, d), "vbar": (B, H, nb, d),
-            "kmean": (B, H, d), "kcov": (B, H, d, d), "mu": (B, H, nb), "sigma": (B, H, nb),
+            "kmean": (B, H, d), "kcov": (B, H, d, d),
         }[name]
         off = getattr(self.struct, name) - self.buffer.data_ptr()
         n = math.prod(dims)
@@ -84,7 +84,7 @@ class PooledStats:
 
 
 def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stats: PooledStats | None = None) -> PooledStats:
-    """Block means of q, k, v and the key mean/covariance, mu and sigma (solattn_pool)."""
+    """Block means of q, k, v and the mean and covariance of the pooled keys (solattn_pool)."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     if stats is None:

@@ -36,7 +36,7 @@ MAX_TOKENS = 262144
 class PooledStruct(ctypes.Structure):
     """Mirror of solattn_pooled_t."""
 
-    _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov", "mu", "sigma")]
+    _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov")]
 
 
 _lib = None

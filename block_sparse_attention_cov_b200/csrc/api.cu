@@ -41,7 +41,7 @@ int check_qkv(const void* q, const void* k, const void* v) {
 
 int check_pooled(const solattn_pooled_t* p) {
   if (!p) return SOLATTN_ERR_ARG;
-  const void* ptrs[7] = {p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, p->mu, p->sigma};
+  const void* ptrs[5] = {p->qbar, p->kbar, p->vbar, p->kmean, p->kcov};
   for (const void* x : ptrs)
     if (!x) return SOLATTN_ERR_ARG;
   for (const void* x : ptrs)
@@ -69,7 +69,7 @@ int current_device_sms(int* sms) {
 }
 
 PooledPtrs to_ptrs(const solattn_pooled_t* p) {
-  return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, p->mu, p->sigma};
+  return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov};
 }
 
 int run_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
@@ -139,10 +139,10 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t nb = (static_cast<size_t>(N) + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
   const size_t f = sizeof(float);
-  const size_t sizes[7] = {bh * nb * d * f, bh * nb * d * f, bh * nb * d * f, bh * d * f,
-                           bh * static_cast<size_t>(d) * d * f, bh * nb * f, bh * nb * f};
-  size_t off[7], total = 0;
-  for (int i = 0; i < 7; ++i) {
+  const size_t sizes[5] = {bh * nb * d * f, bh * nb * d * f, bh * nb * d * f, bh * d * f,
+                           bh * static_cast<size_t>(d) * d * f};
+  size_t off[5], total = 0;
+  for (int i = 0; i < 5; ++i) {
     off[i] = total;
     total += round256(sizes[i]);
   }
@@ -155,8 +155,6 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
     pooled->vbar = reinterpret_cast<float*>(b + off[2]);
     pooled->kmean = reinterpret_cast<float*>(b + off[3]);
     pooled->kcov = reinterpret_cast<float*>(b + off[4]);
-    pooled->mu = reinterpret_cast<float*>(b + off[5]);
-    pooled->sigma = reinterpret_cast<float*>(b + off[6]);
   } else if (pooled && !base) {
     return SOLATTN_ERR_ARG;
   }

@@ -103,6 +103,8 @@ struct __align__(1024) Smem {
   float cmax[2][2];                  // reference max of the correction (natural units)
   int unit[2];
   int count[2];
+  float rq[2][D];                    // routing: qbar of the unit's two query blocks
+  float rstat[4][4];                 // routing: per-warp partial mu / quadratic form sums
   float rscore[2][kChunk];           // proxy scores of the chunk being routed
   float rweight[2][kChunk];          // correction weights n_j e^{s_hat - M} (0 if kept)
   float rscale[2];                   // rescale of the running correction sums
@@ -136,8 +138,8 @@ struct Params {
   const float* qbar;
   const float* kbar;
   const float* vbar;
-  const float* mu;
-  const float* sigma;
+  const float* kmean;
+  const float* kcov;
   float beta;
   int BH, N, NB, npairs, units;
   DeviceStatus* status;
@@ -197,19 +199,67 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     q1[e] = has1 ? qb[static_cast<long long>(i1) * D + lane * VPL + e] : 0.f;
   }
   const float beta = P.beta;
-  // tau_i = mu_i + beta sigma_i. sigma_i = 0 means a constant proxy row (every
-  // score equals mu_i = tau_i): nothing is strictly above it, so no block is
-  // kept, whatever rounding does to the individual scores.
-  auto tau_of = [&](int i) -> float {
-    if (beta == -INFINITY) return -INFINITY;
-    if (beta == INFINITY) return INFINITY;
-    const float sg = P.sigma[static_cast<long long>(bh) * NB + i];
-    if (sg == 0.f) return INFINITY;
-    return P.mu[static_cast<long long>(bh) * NB + i] + beta * sg;
-  };
-  const float tau0 = tau_of(i0);
-  const float tau1 = has1 ? tau_of(i1) : INFINITY;
   const float scale = rsqrtf(static_cast<float>(D));
+  // tau_i = mu_i + beta sigma_i with mu_i = s qbar_i . kmean and
+  // sigma_i = s sqrt(qbar_i^T C qbar_i), from the head's key mean and covariance
+  // (the proxy row itself is never formed). sigma_i = 0 means a constant proxy
+  // row (every score equals mu_i = tau_i): nothing is strictly above it, so no
+  // block is kept, whatever rounding does to the individual scores.
+  float tau0 = beta, tau1 = has1 ? beta : INFINITY;
+  if (beta != -INFINITY && beta != INFINITY) {
+    // D = 128: thread rt owns column rt of both blocks; D = 64: column rt % 64
+    // of block rt / 64. y_b[c] = sum_r C[r][c] qbar_b[r] (C is symmetric).
+    const int col = rt % D, b1 = rt / D;
+    const float* C = P.kcov + static_cast<long long>(bh) * D * D;
+    if constexpr (D == 128) {
+      sm.rq[0][rt] = qb[static_cast<long long>(i0) * D + rt];
+      sm.rq[1][rt] = has1 ? qb[static_cast<long long>(i1) * D + rt] : 0.f;
+    } else {
+      sm.rq[rt / 64][col] = (rt < 64 || has1) ? qb[static_cast<long long>(i0 + rt / 64) * D + col] : 0.f;
+    }
+    named_bar_sync(1, 128);
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll 16
+    for (int r = 0; r < D; ++r) {
+      const float c = __ldg(C + r * D + col);
+      if constexpr (D == 128) {
+        y0 = fmaf(sm.rq[0][r], c, y0);
+        y1 = fmaf(sm.rq[1][r], c, y1);
+      } else {
+        y0 = fmaf(sm.rq[b1][r], c, y0);
+      }
+    }
+    const float km = __ldg(P.kmean + static_cast<long long>(bh) * D + col);
+    float part[4];  // mu_0, quad_0, mu_1, quad_1 (partial over this thread's column)
+    if constexpr (D == 128) {
+      part[0] = sm.rq[0][col] * km;
+      part[1] = sm.rq[0][col] * y0;
+      part[2] = sm.rq[1][col] * km;
+      part[3] = sm.rq[1][col] * y1;
+    } else {
+      const float m = sm.rq[b1][col] * km, qd = sm.rq[b1][col] * y0;
+      part[0] = b1 == 0 ? m : 0.f;
+      part[1] = b1 == 0 ? qd : 0.f;
+      part[2] = b1 == 1 ? m : 0.f;
+      part[3] = b1 == 1 ? qd : 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part[x] += __shfl_xor_sync(0xffffffffu, part[x], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x) sm.rstat[rw][x] = part[x];
+    }
+    named_bar_sync(1, 128);
+    float tot[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) tot[x] = (sm.rstat[0][x] + sm.rstat[1][x]) + (sm.rstat[2][x] + sm.rstat[3][x]);
+    const float sg0 = scale * sqrtf(fmaxf(tot[1], 0.f)), sg1 = scale * sqrtf(fmaxf(tot[3], 0.f));
+    tau0 = sg0 == 0.f ? INFINITY : scale * tot[0] + beta * sg0;
+    tau1 = (!has1 || sg1 == 0.f) ? INFINITY : scale * tot[2] + beta * sg1;
+  }
   const int nlast = P.N - (NB - 1) * kBN;
   if (rt < 2) {
     sm.rmax[rt] = -INFINITY;
@@ -979,8 +1029,8 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
   p.qbar = a.pooled.qbar;
   p.kbar = a.pooled.kbar;
   p.vbar = a.pooled.vbar;
-  p.mu = a.pooled.mu;
-  p.sigma = a.pooled.sigma;
+  p.kmean = a.pooled.kmean;
+  p.kcov = a.pooled.kcov;
   p.beta = a.beta;
   p.BH = a.BH;
   p.N = a.N;

@@ -13,8 +13,6 @@ struct PooledPtrs {
   float* vbar;
   float* kmean;
   float* kcov;
-  float* mu;
-  float* sigma;
 };
 
 struct ForwardArgs {

@@ -7,13 +7,14 @@
 // deviation come from the mean of the pooled keys and their d x d second-moment
 // matrix, without forming the row ("Una soglia per ogni riga", last paragraph).
 //
-// Three launches:
+// Two launches:
 //   pool_means_kernel  -- HBM-bound: reads q, k, v once with 128-bit loads and
 //                         writes the fp32 block means (qbar, kbar, vbar).
 //   key_stats_kernel   -- per head: mean of kbar and its covariance (two-pass,
-//                         divided by N_b), one 32x32 tile (and its mirror) per CTA.
-//   row_stats_kernel   -- per query block: mu_i = s qbar_i . kmean and
-//                         sigma_i = s sqrt(max(0, qbar_i^T C qbar_i)), 64 blocks per CTA.
+//                         divided by N_b), one cluster of CTAs per head.
+// The per-row statistics mu_i, sigma_i are evaluated by the forward kernel's
+// routing warps from kmean and kcov.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -102,150 +103,146 @@ __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restr
   }
 }
 
-// Covariance of the pooled keys, two-pass. grid = (number of 32x32 tiles on or
-// above the diagonal, BH); CTA (ta <= tb) computes tile (ta, tb) and writes it
-// and its mirror (tb, ta). Pass 1: mean of the 64 columns it needs (fixed
-// order); pass 2: sum over key blocks of the deviations' outer products, 64
-// key blocks staged in shared memory per trip.
-template <int D>
-__global__ void __launch_bounds__(256) key_stats_kernel(const float* __restrict__ kbar, float* __restrict__ kmean,
-                                                        float* __restrict__ kcov, int NB) {
-  constexpr int T = D / 32;
-  constexpr int JC = 128;
-  __shared__ float mpart[8][64];
-  __shared__ float mcol[64];        // means of columns ta*32.. (0-31) and tb*32.. (32-63)
-  __shared__ float da[JC][33];      // deviations, padded against bank conflicts
-  __shared__ __align__(16) float db[JC][32];
-  const int tid = threadIdx.x;
-  const int bh = blockIdx.y;
-  int ta = 0, tb = 0;
-  {  // blockIdx.x -> (ta, tb), ta <= tb, row-major over the upper triangle
-    int rem = blockIdx.x;
-    for (ta = 0; ta < T; ++ta) {
-      if (rem < T - ta) { tb = ta + rem; break; }
-      rem -= T - ta;
-    }
-  }
-  const float* kb = kbar + static_cast<long long>(bh) * NB * D;
-  {
-    // 4 partial sums per column, each over rows part, part + 4, ...; 8
-    // independent accumulators keep 8 loads in flight (fixed summation order)
-    const int c = tid % 64, part = tid / 64;
-    const int col = c < 32 ? ta * 32 + c : tb * 32 + (c - 32);
-    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int j = part;
-    for (; j + 28 < NB; j += 32) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc8[u] += kb[static_cast<long long>(j + 4 * u) * D + col];
-    }
-    for (int u = 0; j < NB; j += 4, ++u) acc8[u & 7] += kb[static_cast<long long>(j) * D + col];
-    mpart[part][c] = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-  }
-  __syncthreads();
-  if (tid < 64) {
-    mcol[tid] = ((mpart[0][tid] + mpart[1][tid]) + (mpart[2][tid] + mpart[3][tid])) / static_cast<float>(NB);
-    if (ta == tb && tid < 32) kmean[static_cast<long long>(bh) * D + ta * 32 + tid] = mcol[tid];
-  }
-  __syncthreads();
-  const int a = tid / 8, b0 = (tid % 8) * 4;  // this thread: row a, columns b0..b0+3 of the tile
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int j0 = 0; j0 < NB; j0 += JC) {
-    for (int e = tid; e < JC * 32; e += 256) {
-      const int jj = e / 32, cc = e % 32, j = j0 + jj;
-      const bool ok = j < NB;
-      da[jj][cc] = ok ? kb[static_cast<long long>(j) * D + ta * 32 + cc] - mcol[cc] : 0.f;
-      db[jj][cc] = ok ? kb[static_cast<long long>(j) * D + tb * 32 + cc] - mcol[32 + cc] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int jj = 0; jj < JC; ++jj) {
-      const float x = da[jj][a];
-      const float4 y = *reinterpret_cast<const float4*>(&db[jj][b0]);
-      acc[0] = fmaf(x, y.x, acc[0]);
-      acc[1] = fmaf(x, y.y, acc[1]);
-      acc[2] = fmaf(x, y.z, acc[2]);
-      acc[3] = fmaf(x, y.w, acc[3]);
-    }
-    __syncthreads();
-  }
-  const float inv = 1.f / static_cast<float>(NB);
-  float* out = kcov + static_cast<long long>(bh) * D * D;
-  const int row = ta * 32 + a, col = tb * 32 + b0;
-  *reinterpret_cast<float4*>(out + static_cast<long long>(row) * D + col) =
-      make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  if (ta != tb) {
-#pragma unroll
-    for (int x = 0; x < 4; ++x) out[static_cast<long long>(col + x) * D + row] = acc[x] * inv;
-  }
-}
+// Mean and covariance of the pooled keys of one head, two-pass, by a cluster of
+// kSplit CTAs (one per contiguous slice of key blocks), 256 threads each:
+//   1. every CTA sums its slice's columns; the cluster exchanges the kSplit
+//      partial sums through distributed shared memory and every CTA forms the
+//      same mean (fixed order);
+//   2. every CTA accumulates the outer products of its slice's deviations
+//      (kbar_j - mean) into a D x D partial, staged 32 key blocks at a time;
+//   3. CTA r adds the kSplit partials of rows r*D/kSplit.. in rank order and
+//      writes them divided by N_b. The summation order is fixed: every call
+//      gives the same bits.
+// Thread (ta, tb) of step 2 owns rows {4 ta + e, 64 + 4 ta + e} and columns
+// {4 tb + e, 64 + 4 tb + e} (D = 128; D = 64: the first set only), so the
+// float4 reads of a staged row by one quarter-warp touch 128 contiguous bytes.
+constexpr int kSplit = 8;   // CTAs per head (portable cluster size)
+constexpr int kRows = 32;   // key blocks staged per trip
 
-// mu_i = s qbar_i . kmean and sigma_i = s sqrt(max(0, qbar_i^T C qbar_i)) for 64
-// query blocks per CTA: thread t owns block t / 4 and a quarter of the columns
-// of y = C qbar (C symmetric), then reduces qbar . y over the 4 threads.
-// grid = (ceil(NB / 64), BH); dynamic smem = C (D*D) + 64 padded qbar rows.
 template <int D>
-__global__ void __launch_bounds__(256) row_stats_kernel(const float* __restrict__ qbar,
-                                                        const float* __restrict__ kmean,
-                                                        const float* __restrict__ kcov, float* __restrict__ mu,
-                                                        float* __restrict__ sigma, int NB) {
-  constexpr int QS = D + 4;     // padded row stride of the staged qbar rows
-  constexpr int CW = D / 4;     // columns per thread
-  extern __shared__ __align__(16) float smem_f[];
-  float* C = smem_f;            // [D][D]
-  float* Q = C + D * D;         // [64][QS]
-  float* km = Q + 64 * QS;      // [D]
+struct KeyStatsSmem {
+  float part[D][D];         // this CTA's sum of deviation outer products
+  float dev[kRows][D];      // staged deviations
+  float colpart[256 / (D / 4)][D];
+  float csum[D];            // this CTA's column sums (read by the whole cluster)
+  float mean[D];
+};
+
+template <int D>
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(256)
+    key_stats_kernel(const float* __restrict__ kbar, float* __restrict__ kmean, float* __restrict__ kcov, int NB) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(16) unsigned char ks_raw[];
+  KeyStatsSmem<D>& sm = *reinterpret_cast<KeyStatsSmem<D>*>(ks_raw);
+  cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x;
+  const int rank = static_cast<int>(cluster.block_rank());
   const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * 64;
-  const float* cg = kcov + static_cast<long long>(bh) * D * D;
-  for (int e = tid; e < D * D / 4; e += 256)
-    reinterpret_cast<float4*>(C)[e] = reinterpret_cast<const float4*>(cg)[e];
-  for (int e = tid; e < 64 * D; e += 256) {
-    const int r = e / D, c = e % D;
-    Q[r * QS + c] = (i0 + r < NB) ? qbar[(static_cast<long long>(bh) * NB + i0 + r) * D + c] : 0.f;
+  const int per = (NB + kSplit - 1) / kSplit;
+  const int j0 = min(NB, rank * per), j1 = min(NB, j0 + per);
+  const float* kb = kbar + static_cast<long long>(bh) * NB * D;
+
+  // ---- 1. column sums of the slice, then the head mean
+  {
+    constexpr int C4 = D / 4, RL = 256 / C4;
+    const int c4 = tid % C4, rl = tid / C4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    int j = j0 + rl;
+    for (; j + RL < j1; j += 2 * RL) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(j) * D) + c4);
+      const float4 y = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(j + RL) * D) + c4);
+      a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+      b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    }
+    if (j < j1) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(j) * D) + c4);
+      a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+    }
+    *reinterpret_cast<float4*>(&sm.colpart[rl][c4 * 4]) = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    __syncthreads();
+    if (tid < D) {
+      float t = 0.f;
+#pragma unroll
+      for (int r = 0; r < RL; ++r) t += sm.colpart[r][tid];
+      sm.csum[tid] = t;
+    }
   }
-  if (tid < D) km[tid] = kmean[static_cast<long long>(bh) * D + tid];
+  cluster.sync();
+  if (tid < D) {
+    float t = 0.f;
+    for (int r = 0; r < kSplit; ++r) t += cluster.map_shared_rank(sm.csum, r)[tid];
+    sm.mean[tid] = t / static_cast<float>(NB);
+  }
   __syncthreads();
-  // thread (r, c4): columns c4 * 4 + 16 m .. + 3 (m < D / 16): the four threads
-  // of a row read 64 contiguous bytes of C per step (no bank conflicts)
-  const int r = tid / 4, c4 = tid % 4;
-  const float* qrow = Q + r * QS;
-  float y[CW];
+
+  // ---- 2. sum of the deviations' outer products over the slice
+  constexpr int TT = D / 16;  // rows (and columns) per thread: 8 or 4
+  const int ta = tid / 16, tb = tid % 16;
+  float acc[TT][TT];
 #pragma unroll
-  for (int c = 0; c < CW; ++c) y[c] = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < D; ++k) {
-    const float qk = qrow[k];
-    const float* crow = C + k * D + c4 * 4;
+  for (int x = 0; x < TT; ++x)
 #pragma unroll
-    for (int m = 0; m < CW / 4; ++m) {
-      const float4 cv = *reinterpret_cast<const float4*>(crow + 16 * m);
-      y[4 * m] = fmaf(qk, cv.x, y[4 * m]);
-      y[4 * m + 1] = fmaf(qk, cv.y, y[4 * m + 1]);
-      y[4 * m + 2] = fmaf(qk, cv.z, y[4 * m + 2]);
-      y[4 * m + 3] = fmaf(qk, cv.w, y[4 * m + 3]);
+    for (int y = 0; y < TT; ++y) acc[x][y] = 0.f;
+  for (int c0 = j0; c0 < j1; c0 += kRows) {
+    const int nr = min(kRows, j1 - c0);
+    for (int e = tid; e < kRows * D / 4; e += 256) {
+      const int r = e / (D / 4), c = (e % (D / 4)) * 4;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nr) {
+        x = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(c0 + r) * D + c));
+        x.x -= sm.mean[c]; x.y -= sm.mean[c + 1]; x.z -= sm.mean[c + 2]; x.w -= sm.mean[c + 3];
+      }
+      *reinterpret_cast<float4*>(&sm.dev[r][c]) = x;
     }
-  }
-  float quad = 0.f, dot = 0.f;
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      float av[TT], bv[TT];
 #pragma unroll
-  for (int m = 0; m < CW / 4; ++m) {
+      for (int h = 0; h < TT / 4; ++h) {
+        const float4 x = *reinterpret_cast<const float4*>(&sm.dev[r][64 * h + 4 * ta]);
+        const float4 y = *reinterpret_cast<const float4*>(&sm.dev[r][64 * h + 4 * tb]);
+        av[4 * h] = x.x; av[4 * h + 1] = x.y; av[4 * h + 2] = x.z; av[4 * h + 3] = x.w;
+        bv[4 * h] = y.x; bv[4 * h + 1] = y.y; bv[4 * h + 2] = y.z; bv[4 * h + 3] = y.w;
+      }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = c4 * 4 + 16 * m + e;
-      quad = fmaf(qrow[c], y[4 * m + e], quad);
-      dot = fmaf(qrow[c], km[c], dot);
+      for (int x = 0; x < TT; ++x)
+#pragma unroll
+        for (int y = 0; y < TT; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
+    __syncthreads();
   }
-  quad += __shfl_xor_sync(0xffffffffu, quad, 1);
-  dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-  quad += __shfl_xor_sync(0xffffffffu, quad, 2);
-  dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-  const int i = i0 + r;
-  if ((tid % 4) == 0 && i < NB) {
-    const float s = rsqrtf(static_cast<float>(D));
-    mu[static_cast<long long>(bh) * NB + i] = s * dot;
-    sigma[static_cast<long long>(bh) * NB + i] = s * sqrtf(fmaxf(quad, 0.f));
+#pragma unroll
+  for (int x = 0; x < TT; ++x) {
+    const int row = 64 * (x / 4) + 4 * ta + x % 4;
+#pragma unroll
+    for (int h = 0; h < TT / 4; ++h)
+      *reinterpret_cast<float4*>(&sm.part[row][64 * h + 4 * tb]) =
+          make_float4(acc[x][4 * h], acc[x][4 * h + 1], acc[x][4 * h + 2], acc[x][4 * h + 3]);
   }
+  cluster.sync();
+
+  // ---- 3. rows rank * D / kSplit .. of the covariance: partials in rank order
+  {
+    constexpr int R = D / kSplit;          // rows per CTA: 16 or 8
+    constexpr int V4 = R * D / 4 / 256;    // float4 per thread: 2 or 1 (D = 64: 128 threads idle)
+    const float inv = 1.f / static_cast<float>(NB);
+    float* out = kcov + static_cast<long long>(bh) * D * D + static_cast<long long>(rank) * R * D;
+#pragma unroll
+    for (int v = 0; v < (V4 > 0 ? V4 : 1); ++v) {
+      const int e = tid + 256 * v;
+      if (e < R * D / 4) {
+        const int row = rank * R + e / (D / 4), c = (e % (D / 4)) * 4;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < kSplit; ++r) {
+          const float4 y = *reinterpret_cast<const float4*>(&cluster.map_shared_rank(&sm.part[0][0], r)[row * D + c]);
+          t.x += y.x; t.y += y.y; t.z += y.z; t.w += y.w;
+        }
+        reinterpret_cast<float4*>(out)[e] = make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+      }
+    }
+    if (rank == 0 && tid < D) kmean[static_cast<long long>(bh) * D + tid] = sm.mean[tid];
+  }
+  cluster.sync();  // no CTA leaves while another still reads its shared memory
 }
 
 template <int D>
@@ -257,15 +254,10 @@ cudaError_t launch_pool_d(const uint16_t* q, const uint16_t* k, const uint16_t* 
   pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, BH, N, NB);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  constexpr int T = D / 32;
-  key_stats_kernel<D><<<dim3(T * (T + 1) / 2, BH), 256, 0, stream>>>(p.kbar, p.kmean, p.kcov, NB);
-  e = cudaGetLastError();
+  const int smem = static_cast<int>(sizeof(KeyStatsSmem<D>));
+  e = cudaFuncSetAttribute(key_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const size_t smem = (static_cast<size_t>(D) * D + 64 * (D + 4) + D) * sizeof(float);
-  e = cudaFuncSetAttribute(row_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  row_stats_kernel<D><<<dim3((NB + 63) / 64, BH), 256, smem, stream>>>(p.qbar, p.kmean, p.kcov, p.mu, p.sigma, NB);
+  key_stats_kernel<D><<<dim3(kSplit, BH), 256, smem, stream>>>(p.kbar, p.kmean, p.kcov, NB);
   return cudaGetLastError();
 }
 

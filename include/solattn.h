@@ -63,11 +63,9 @@ enum solattn_status_code {
  *   qbar, kbar, vbar  [B][H][N_b][d]  block means over valid tokens
  *   kmean             [B][H][d]       mean of the pooled keys (each block counts once)
  *   kcov              [B][H][d][d]    covariance of the pooled keys, divided by N_b
- *   mu, sigma         [B][H][N_b]     mean and population standard deviation of
- *                                     every proxy row s_hat_i. (paithon.it,
- *                                     "Una soglia per ogni riga": the threshold's
- *                                     statistics come from the key mean and the
- *                                     d x d second-moment matrix.)
+ * (paithon.it, "Una soglia per ogni riga", last paragraph: the mean and the
+ * d x d second-moment matrix of the pooled keys give every proxy row's mean and
+ * spread; solattn_forward evaluates them per query block from kmean and kcov.)
  */
 typedef struct {
   float* qbar;
@@ -75,8 +73,6 @@ typedef struct {
   float* vbar;
   float* kmean;
   float* kcov;
-  float* mu;
-  float* sigma;
 } solattn_pooled_t;
 
 /*
@@ -91,14 +87,14 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
 /*
  * Pooling (paithon.it, "Perché l'attenzione pesa tanto nei video": proxy scores
  * are products of block-mean queries and keys; "Una soglia per ogni riga",
- * last paragraph: mu_i and sigma_i from the mean and d x d second-moment matrix
- * of the pooled keys).
+ * last paragraph: the row statistics come from the mean and d x d
+ * second-moment matrix of the pooled keys).
  * Reads q, k, v once and writes every array of `pooled` (the struct itself is
  * host memory, its pointers are device memory):
  *   qbar_i = mean of the valid query tokens of block i (likewise kbar, vbar);
  *   kmean  = (1/N_b) sum_j kbar_j;
- *   kcov   = (1/N_b) sum_j (kbar_j - kmean)(kbar_j - kmean)^T;
- *   mu_i   = s qbar_i . kmean;   sigma_i = s sqrt(max(0, qbar_i^T kcov qbar_i)).
+ *   kcov   = (1/N_b) sum_j (kbar_j - kmean)(kbar_j - kmean)^T  (two-pass, fp32,
+ *            fixed summation order: the result is the same on every call).
  */
 int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                  const solattn_pooled_t* pooled, void* stream);
@@ -111,7 +107,12 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
  * attended exactly, skipped blocks approximated by the zeroth-order Taylor term
  * that reuses their proxy scores, both in the same softmax state).
  *
- * For every query token t of block i, with s_hat_ij = s qbar_i . kbar_j:
+ * For every query block i, with s = 1/sqrt(d) and s_hat_ij = s qbar_i . kbar_j,
+ * the row statistics are evaluated in the routing warps from kmean and kcov:
+ *   mu_i = s qbar_i . kmean,  sigma_i = s sqrt(max(0, qbar_i^T kcov qbar_i)),
+ *   tau_i = mu_i + beta sigma_i  (tau_i = +inf when sigma_i = 0: a constant row
+ *   has no block strictly above its mean).
+ * For every query token t of block i:
  *   out_t = (sum_{j in S_i} sum_{u in j} e^{s q_t.k_u} v_u + sum_{j not in S_i} n_j e^{s_hat_ij} vbar_j)
  *         / (sum_{j in S_i} sum_{u in j} e^{s q_t.k_u}     + sum_{j not in S_i} n_j e^{s_hat_ij})
  *   lse_t = natural log of the denominator;   density_out_i = |S_i|.

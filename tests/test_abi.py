@@ -71,7 +71,7 @@ def test_forward_argument_errors(L):
     assert _fwd(L, k=ctypes.c_void_p(0x7F0000000008)) == _lib.ERR_ALIGN
     assert _fwd(L, lse=ctypes.c_void_p(0x7F0000000002)) == _lib.ERR_ALIGN
     bad = _pooled_struct()
-    bad.mu = None
+    bad.kmean = None
     assert _fwd(L, pooled=bad) == _lib.ERR_ARG
     bad = _pooled_struct()
     bad.kcov = 0x100004
@@ -96,13 +96,13 @@ def test_pooled_layout_sizes_and_alignment(L):
     assert L.solattn_pooled_layout(B, H, N, d, None, None, ctypes.byref(n)) == 0
     nb = math.ceil(N / 64)
     r = lambda x: (x + 255) // 256 * 256
-    want = 3 * r(B * H * nb * d * 4) + r(B * H * d * 4) + r(B * H * d * d * 4) + 2 * r(B * H * nb * 4)
+    want = 3 * r(B * H * nb * d * 4) + r(B * H * d * 4) + r(B * H * d * d * 4)
     assert n.value == want
     st = _lib.PooledStruct()
     base = 0x10000000
     assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base), ctypes.byref(st), None) == 0
     ptrs = [getattr(st, f) for f, _ in _lib.PooledStruct._fields_]
     assert ptrs[0] == base and all(p % 256 == 0 for p in ptrs) and ptrs == sorted(ptrs)
-    assert ptrs[-1] + r(B * H * nb * 4) == base + want
+    assert ptrs[-1] + r(B * H * d * d * 4) == base + want
     assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base + 8), ctypes.byref(st), None) == _lib.ERR_ALIGN
     assert L.solattn_pooled_layout(B, H, N, 80, None, None, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED

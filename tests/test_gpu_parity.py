@@ -69,7 +69,8 @@ def _wl(B, H, d, N):
 
 
 # --------------------------------------------------------------------------- pooling
-@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], WORKLOADS["mid"], _wl(2, 3, 128, 1000), _wl(1, 2, 64, 37)],
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], WORKLOADS["mid"], _wl(2, 3, 128, 1000), _wl(1, 2, 64, 37),
+                                _wl(1, 1, 128, 75600), _wl(1, 1, 64, 262144)],
                          ids=lambda w: w.name)
 def test_pool_matches_oracle(wl):
     q, k, v = make_qkv(wl, seed=1)
@@ -85,8 +86,6 @@ def test_pool_matches_oracle(wl):
             np.testing.assert_allclose(st.view("vbar")[b, h].cpu().numpy(), orc.pool(vv), rtol=1e-5, atol=1e-6)
             np.testing.assert_allclose(st.view("kmean")[b, h].cpu().numpy(), r["kmean"], rtol=1e-5, atol=1e-6)
             np.testing.assert_allclose(st.view("kcov")[b, h].cpu().numpy(), r["kcov"], rtol=1e-4, atol=1e-6)
-            np.testing.assert_allclose(st.view("mu")[b, h].cpu().numpy(), r["mu"], rtol=1e-4, atol=1e-6)
-            np.testing.assert_allclose(st.view("sigma")[b, h].cpu().numpy(), r["sigma"], rtol=1e-4, atol=1e-6)
 
 
 # --------------------------------------------------------------------------- forward
