@@ -11,23 +11,21 @@
 // the SM.
 //
 // Work unit: two adjacent 64-token query blocks (128 rows, the full-rate
-// tcgen05 tile height) of one head. The key tiles of a unit are the union of
-// the two blocks' kept sets; a tile kept by only one of the two blocks is still
-// multiplied for all 128 rows, and the other block's rows mask it out (their P
-// row is zero and their softmax state is untouched), so each block's result is
-// exactly its own.
+// tcgen05 tile height) of one head. The key blocks of a unit are the union of
+// the two blocks' kept sets, taken two at a time as 128-key tiles (any two
+// kept blocks, not only neighbours); a block kept by only one of the two
+// query blocks is still multiplied for all 128 rows, and the other block's
+// rows mask it out (their P is zero and their softmax state is untouched), so
+// each block's result is exactly its own.
 //
-// One persistent CTA per SM, 320 threads, warp roles:
-//   warps 0-3  softmax / epilogue: thread r owns row r of the unit (TMEM lane r)
-//   warps 4-7  routing, one unit ahead: fetch the next unit from the atomic
-//              scheduler, copy its Q rows into TMEM, score every key block,
-//              build the ordered kept list and the correction sums in shared
-//              memory (double-buffered unit slots)
-//   warp 8     TMA producer: K and V tiles of the kept list only
-//   warp 9     MMA issuer (one thread): S = Q K^T and O += P V with A (Q, P)
-//              in TMEM and B (K, V) in shared memory
-// TMEM columns: Q slot 0/1 at 0/64, O at 128, S buffers at 256/320, P buffers
-// at 384/416 (512 allocated).
+// One persistent CTA per SM, 512 threads (roles at the kernel below). S = Q K^T
+// runs with both operands in shared memory (Q tile 128 x d, K tile 128 x d:
+// at N = 128 the operand traffic fits the shared-memory bandwidth), O += P V
+// with P in TMEM (written over its own S) and V in shared memory. Three S
+// slots let the QKs of the next two tiles run while the softmax works on one;
+// eight softmax warps split every 128-key tile in two 64-key halves (two warps
+// per row group, agreeing on the row max), so two warps share each SM
+// sub-partition's exponential unit.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cmath>
@@ -55,21 +53,13 @@ __device__ unsigned long long g_trace[40][4096];
 namespace {
 
 constexpr int kBM = 128;      // rows per unit
-constexpr int kBN = 64;       // keys per tile (one block)
-constexpr int kStages = 5;    // depth of the K ring and of the V ring
+constexpr int kBN = 64;       // keys per block (a tile holds two)
 constexpr int kNbMax = 4096;  // key blocks per head supported
-constexpr int kThreads = 512;
-// Registers per thread after rebalancing (launched with 65536 / 512 = 128):
-// 2 softmax warpgroups x 136 + routing 120 + producer/MMA 120, times 128 threads
-// each = 65536.
-constexpr int kRegsSoftmax = 136, kRegsRouting = 120, kRegsIssue = 120;
-static_assert(128 * (2 * kRegsSoftmax + kRegsRouting + kRegsIssue) <= 65536, "register split exceeds the launch");
+constexpr int kThreads = 512;  // 16 warps, 128 registers per thread
 constexpr int kChunk = 16;    // pooled key blocks per routing chunk (4 per routing warp)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.0f;  // log2 units a row max may grow before O is rescaled
-
-constexpr uint32_t kColQ = 0, kColS = 64, kColP = 192, kColO = 256;  // + group * 64 / 32 / 128
 
 // Wait-site ids reported in the status word when a bounded wait gives up.
 enum : uint32_t {
@@ -90,14 +80,22 @@ enum : uint32_t {
   kSiteRouteChunk,
   kSiteQFree,
   kSiteBDone,
+  kSiteQFull,
+  kSiteMlReady,
+  kSitePvDone,
 };
 
 template <int D>
 struct __align__(1024) Smem {
-  uint8_t kt[kStages][kBN * D * 2];  // SW128 K tiles (1024-aligned: size is a multiple of 8 KB)
-  uint8_t vt[kStages][kBN * D * 2];  // SW128 V tiles
-  float rchunk[2][2][kChunk][D];     // routing: [buffer][kbar | vbar][key block][column]
-  uint16_t list[2][kNbMax];          // kept (union) list: j | keep-bits << 14
+  // K ring: one stage per 128-key tile (two blocks stacked in every 64-column
+  // panel, as one N = 128 operand); V ring: one stage per block. Sizes are
+  // multiples of 1 KB, so every stage stays 1024-aligned for the swizzle.
+  static constexpr int kKStages = D == 128 ? 3 : 4;
+  static constexpr int kVStages = D == 128 ? 4 : 8;
+  uint8_t qt[kBM * D * 2];               // Q tile of the unit, SW128 K-major panels of 128 rows
+  uint8_t kt[kKStages][kBM * D * 2];     // K tiles, same layout
+  uint8_t vt[kVStages][kBN * D * 2];     // V blocks, SW128 panels of 64 rows
+  float rchunk[2][kChunk][D];        // routing: pooled keys of a chunk, double-buffered
   float cnum[2][2][D];               // correction numerator per slot and block
   float cden[2][2];
   float cmax[2][2];                  // reference max of the correction (natural units)
@@ -111,15 +109,19 @@ struct __align__(1024) Smem {
   float rmax[2];                     // running max of the skipped proxy scores
   float rden[2];                     // running correction denominators
   int rkept[2];                      // running kept counts
-  uint32_t bits[2][kNbMax / 32];     // kept bitmaps of the unit being routed
-  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_full[2];  // per softmax group
-  uint64_t o_free, b_done, q_free;
+  uint32_t bits[2][2][kNbMax / 32];  // kept bitmaps [slot][query block][word]: the unit's key list
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  // Per S slot: QK landed / P stored by all four softmax warps / PV of the
+  // slot's tile completed. Per-slot barriers keep a warp that runs a tile
+  // ahead from arriving on the phase of the tile its neighbours are still on.
+  uint64_t s_full[3], p_full[3], pv_done[3];
+  uint64_t o_free[2];                // per unit slot: the epilogue has read O
+  uint64_t q_full, q_free;
   uint64_t route_full[2], route_empty[2];
   uint64_t rfull[2];                 // routing chunk buffers landed
   uint64_t mma_done[2];
-  float mB[2][kBM];                  // group B's final running max / sum per row, per slot
-  float lB[2][kBM];
+  float xm[kBM][2];                  // softmax: row max of each key half (exchange)
+  float xl[kBM][2];                  // softmax: row sum of each key half (epilogue)
   uint32_t tmem_base;
   int bcast;
   int abort_flag;
@@ -185,11 +187,13 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     const int nk = min(kChunk, NB - j0);
     const uint32_t buf = (chunk_ctr + c) & 1;
     const uint32_t bytes = static_cast<uint32_t>(nk) * D * 4;
-    mbar_arrive_expect_tx(&sm.rfull[buf], 2 * bytes);
-    bulk_copy_g2s(&sm.rchunk[buf][0][0][0], kb + static_cast<long long>(j0) * D, bytes, &sm.rfull[buf]);
-    bulk_copy_g2s(&sm.rchunk[buf][1][0][0], vb + static_cast<long long>(j0) * D, bytes, &sm.rfull[buf]);
+    mbar_arrive_expect_tx(&sm.rfull[buf], bytes);
+    bulk_copy_g2s(&sm.rchunk[buf][0][0], kb + static_cast<long long>(j0) * D, bytes, &sm.rfull[buf]);
   };
   if (rt == 0) issue(0);
+  // pooled values: this thread's column of the chunk's blocks, loaded into
+  // registers at the start of the chunk (D = 128: column rt; D = 64: rt % 64)
+  const int vcol = rt % D;
 
   const float* qb = P.qbar + static_cast<long long>(bh) * NB * D;
   float q0[VPL], q1[VPL];
@@ -277,6 +281,10 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   for (int c = 0; c < nchunks; ++c) {
     const uint32_t g = chunk_ctr + c, buf = g & 1;
     if (rt == 0 && c + 1 < nchunks) issue(c + 1);  // buffer (c+1)&1 was released by chunk c-1
+    float vcur[kChunk];
+#pragma unroll
+    for (int jj = 0; jj < kChunk; ++jj)
+      vcur[jj] = (c * kChunk + jj < NB) ? __ldg(vb + static_cast<long long>(c * kChunk + jj) * D + vcol) : 0.f;
     const bool landed = mbar_wait(&sm.rfull[buf], (g >> 1) & 1, abort_flag, st, kSiteRouteChunk, u);
     if (named_bar_or(1, 128, !landed || *abort_flag)) {
       // aborting: let the copies already issued (chunks c and c + 1) land first
@@ -293,7 +301,7 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     float v[8];
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const float* row = &sm.rchunk[buf][0][rw * 4 + kk][lane * VPL];
+      const float* row = &sm.rchunk[buf][rw * 4 + kk][lane * VPL];
       float x[VPL];
       if constexpr (VPL == 4) {
         const float4 t = *reinterpret_cast<const float4*>(row);
@@ -365,28 +373,27 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
         sm.rmax[b] = mnew;
         sm.rkept[b] += __popc(kmask);
         // two 16-block chunks per 32-bit bitmap word (even chunk first)
-        if (c & 1) sm.bits[b][c >> 1] |= kmask << 16;
-        else sm.bits[b][c >> 1] = kmask;
+        if (c & 1) sm.bits[s][b][c >> 1] |= kmask << 16;
+        else sm.bits[s][b][c >> 1] = kmask;
       }
     }
     named_bar_sync(1, 128);
-    // ---- correction sums: sum_j w_bj vbar_j[col]
+    // ---- correction sums: sum_j w_bj vbar_j[col] (weights of kept and pad blocks are 0)
     {
-      const float* vrows = &sm.rchunk[buf][1][0][0];
       if constexpr (D == 128) {
-        const float sc0 = sm.rscale[0], sc1 = sm.rscale[1];
-        float a0 = acc[0] * sc0, a1 = acc[1] * sc1;
-        for (int jj = 0; jj < nk; ++jj) {
-          const float x = vrows[jj * D + rt];
-          a0 = fmaf(sm.rweight[0][jj], x, a0);
-          a1 = fmaf(sm.rweight[1][jj], x, a1);
+        float a0 = acc[0] * sm.rscale[0], a1 = acc[1] * sm.rscale[1];
+#pragma unroll
+        for (int jj = 0; jj < kChunk; ++jj) {
+          a0 = fmaf(sm.rweight[0][jj], vcur[jj], a0);
+          a1 = fmaf(sm.rweight[1][jj], vcur[jj], a1);
         }
         acc[0] = a0;
         acc[1] = a1;
       } else {
-        const int b = rt / 64, col = rt % 64;
+        const int b = rt / 64;
         float a0 = acc[0] * sm.rscale[b];
-        for (int jj = 0; jj < nk; ++jj) a0 = fmaf(sm.rweight[b][jj], vrows[jj * D + col], a0);
+#pragma unroll
+        for (int jj = 0; jj < kChunk; ++jj) a0 = fmaf(sm.rweight[b][jj], vcur[jj], a0);
         acc[0] = a0;
       }
     }
@@ -408,27 +415,9 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   if (rw == 0) {
     const int nwords = (nchunks + 1) / 2;  // one 32-bit word per two chunks
     int base = 0;
-    for (int w0 = 0; w0 < nwords; w0 += 32) {
-      const int wi = w0 + lane;
-      const uint32_t m0 = wi < nwords ? sm.bits[0][wi] : 0u;
-      const uint32_t m1 = wi < nwords ? sm.bits[1][wi] : 0u;
-      uint32_t un = m0 | m1;
-      const int cnt = __popc(un);
-      int incl = cnt;
+    for (int wi = lane; wi < nwords; wi += 32) base += __popc(sm.bits[s][0][wi] | sm.bits[s][1][wi]);
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      int pos = base + incl - cnt;
-      while (un) {
-        const int bit = __ffs(un) - 1;
-        const uint32_t flags = ((m0 >> bit) & 1u) | (((m1 >> bit) & 1u) << 1);
-        sm.list[s][pos++] = static_cast<uint16_t>((wi * 32 + bit) | (flags << 14));
-        un &= un - 1u;
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
-    }
+    for (int off = 16; off > 0; off >>= 1) base += __shfl_xor_sync(0xffffffffu, base, off);
     if (lane == 0) {
       sm.count[s] = base;
       if (P.density) {
@@ -440,32 +429,34 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   return true;
 }
 
-// Reads the unit's 128 Q rows (bf16 pairs = one 32-bit TMEM column per pair)
-// into registers; rows past N are zero.
-template <int D>
-__device__ __forceinline__ void load_q_rows(const Params& P, int bh, int pair, int rt, uint32_t (&w)[D / 2]) {
-  const int row = pair * kBM + rt;
-  const uint4* src = reinterpret_cast<const uint4*>(P.q + (static_cast<long long>(bh) * P.N + row) * D);
-  const bool ok = row < P.N;
-#pragma unroll
-  for (int x = 0; x < D / 8; ++x) {
-    const uint4 t = ok ? __ldg(src + x) : make_uint4(0, 0, 0, 0);
-    w[4 * x] = t.x; w[4 * x + 1] = t.y; w[4 * x + 2] = t.z; w[4 * x + 3] = t.w;
+// In-order walk over a unit's key list (the union of the two kept bitmaps of a
+// slot; without routing, every block). next() returns j | keep-bits << 14
+// (bit 14: kept by the first query block, bit 15: by the second). Every lane
+// of a warp walks identically. A walk past the last word returns 0 (no keep
+// bits), so a count that disagreed with the bitmaps could not read past them.
+template <bool ROUTE>
+struct KeyWalk {
+  const uint32_t* b0;
+  const uint32_t* b1;
+  int w, pos;
+  uint32_t rem;
+  __device__ __forceinline__ KeyWalk(const uint32_t* x0, const uint32_t* x1) : b0(x0), b1(x1), w(-1), pos(0), rem(0u) {}
+  __device__ __forceinline__ uint32_t next() {
+    if constexpr (!ROUTE) {
+      return static_cast<uint32_t>(pos++) | 0xC000u;
+    } else {
+      while (rem == 0u) {
+        if (w + 1 >= kNbMax / 32) return 0u;
+        ++w;
+        rem = b0[w] | b1[w];
+      }
+      const int bit = __ffs(rem) - 1;
+      rem &= rem - 1u;
+      const uint32_t f = ((b0[w] >> bit) & 1u) | (((b1[w] >> bit) & 1u) << 1);
+      return static_cast<uint32_t>(w * 32 + bit) | (f << 14);
+    }
   }
-}
-
-template <int D>
-__device__ __forceinline__ void store_q_tmem(uint32_t tmem, int rt, const uint32_t (&w)[D / 2]) {
-  const uint32_t taddr = tmem + (static_cast<uint32_t>((rt / 32) * 32) << 16) + kColQ;
-#pragma unroll
-  for (int c = 0; c < D / 64; ++c) {
-    uint32_t x[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) x[e] = w[c * 32 + e];
-    tmem_st32(taddr + c * 32, x);
-  }
-  tmem_wait_st();
-}
+};
 
 // ---------------------------------------------------------------------------
 // Softmax arithmetic of one row and one 64-key tile (log2 domain, lazily
@@ -495,38 +486,26 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
   return d;
 }
 
-// Masks the pad keys of a partial tile and folds the tile's row max into the
-// lazily rescaled running max m (log2 units). Returns whether the row's O and
-// l must be multiplied by `rescale` (= 2^(m_old - m_new)) before this tile.
-__device__ __forceinline__ bool softmax_max(uint32_t (&sv)[32], uint32_t (&sw)[32], int nv, float sl2, float& m,
-                                            float& rescale) {
+// Sets the pad keys of a partial block (only the last block of a head) to -inf.
+__device__ __forceinline__ void mask_tail(uint32_t (&sv)[64], int nv) {
   constexpr uint32_t kNegInf = 0xFF800000u;
-  if (nv < 64) {  // only the last key block of a head can be partial
+  if (nv < 64) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
+    for (int c = 0; c < 64; ++c)
       if (c >= nv) sv[c] = kNegInf;
-      if (c + 32 >= nv) sw[c] = kNegInf;
-    }
   }
+}
+
+// Max over the valid keys of one 64-key block (raw S units); masks the pad keys.
+__device__ __forceinline__ float tile_max(uint32_t (&sv)[64], int nv) {
+  mask_tail(sv, nv);
   float t[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i)
     t[i] = fmax3(fmax3(__uint_as_float(sv[8 * i]), __uint_as_float(sv[8 * i + 1]), __uint_as_float(sv[8 * i + 2])),
                  fmax3(__uint_as_float(sv[8 * i + 3]), __uint_as_float(sv[8 * i + 4]), __uint_as_float(sv[8 * i + 5])),
                  fmaxf(__uint_as_float(sv[8 * i + 6]), __uint_as_float(sv[8 * i + 7])));
-    t[4 + i] = fmax3(fmax3(__uint_as_float(sw[8 * i]), __uint_as_float(sw[8 * i + 1]), __uint_as_float(sw[8 * i + 2])),
-                     fmax3(__uint_as_float(sw[8 * i + 3]), __uint_as_float(sw[8 * i + 4]), __uint_as_float(sw[8 * i + 5])),
-                     fmaxf(__uint_as_float(sw[8 * i + 6]), __uint_as_float(sw[8 * i + 7])));
-  }
-  const float mx = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(fmax3(t[3], t[4], t[5]), t[6], t[7])) * sl2;
-  rescale = 1.f;
-  if (mx > m + kRescaleSlack) {
-    const bool need = m != -INFINITY;
-    if (need) rescale = ex2_approx(m - mx);
-    m = mx;
-    return need;
-  }
-  return false;
+  return fmaxf(fmax3(t[0], t[1], t[2]), fmax3(fmax3(t[3], t[4], t[5]), t[6], t[7]));
 }
 
 // 2^y for two packed fp32 values on the FMA pipe (relieves the MUFU unit):
@@ -565,11 +544,11 @@ __device__ __forceinline__ void exp2_poly2(float y0, float y1, float& p0, float&
 }
 
 // P for 16 consecutive columns (x holds their raw S bits): 8 packed bf16x2
-// words; adds the fp32 probabilities to l. The first 8 - kPolyPairs column
-// pairs use the MUFU ex2, the others the FMA-pipe polynomial.
-__device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, uint64_t nm2, float& l,
+// words; adds the fp32 probabilities to the packed pair of partial sums l2.
+// The first 8 - kPolyPairs column pairs use the MUFU ex2, the others the
+// FMA-pipe polynomial.
+__device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, uint64_t nm2, uint64_t& l2,
                                               uint32_t (&pw)[8]) {
-  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int c = 0; c < 16; c += 2) {
     float y0, y1, p0, p1;
@@ -580,29 +559,35 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
     } else {
       exp2_poly2(y0, y1, p0, p1);
     }
-    if (c & 2) a1 += p0 + p1; else a0 += p0 + p1;
+    l2 = fadd2(l2, f2_from_bits(__float_as_uint(p0), __float_as_uint(p1)));
     pw[c >> 1] = pack_bf16x2(p0, p1);
   }
-  l += a0 + a1;
 }
 
 // ---------------------------------------------------------------------------
 // The kernel. 512 threads = 16 warps:
-//   warps 0-3   softmax group A (even global tiles) + epilogue
-//   warps 4-7   softmax group B (odd global tiles)
-//   warps 8-11  routing, one unit ahead (Q rows into TMEM after the previous
-//               unit's last QK has completed)
-//   warp 12     TMA producer of the K tiles of the kept list
-//   warps 13/15 MMA issuers of group A / group B (one elected lane issues)
-//   warp 14     TMA producer of the V tiles
-// TMEM: Q at 0 (64 columns), S_A/S_B at 64/128, P_A/P_B at 192/224,
-// O_A/O_B at 256/384. Each group keeps its own running max, sum and O; the
-// epilogue merges the two with the skipped-block correction.
+//   warps 0-7   softmax: warp w covers rows 32 (w % 4) .. + 31 of the unit
+//               (TMEM lanes) and key block w / 4 of every 128-key tile; the
+//               two warps of a row group agree on the row max through a
+//               pairwise barrier. At the end of the unit, once its last PV has
+//               completed, the epilogue (O and the row sum merged with the
+//               skipped-block correction, out and lse written)
+//   warps 8-11  routing, one unit ahead; then the unit's Q tile by TMA once
+//               every QK of the previous unit has completed
+//   warp 12     TMA producer of the K tiles (two kept blocks per stage)
+//   warp 13     MMA issuer for QK (one elected lane), up to two tiles ahead
+//   warp 14     TMA producer of the V blocks
+//   warp 15     MMA issuer for PV
+// TMEM: three S slots of 128 fp32 columns at 0 / 128 / 256 (the bf16 P of a
+// tile is written over the first 64 columns of its own S) and O at 384. The
+// QKs of the next two tiles are in flight while the softmax works on one.
 // ---------------------------------------------------------------------------
 template <int D, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
-    solattn_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const Params P) {
+    solattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const Params P) {
+  constexpr int KS = Smem<D>::kKStages, VS = Smem<D>::kVStages;
+  constexpr uint32_t kColO = 3 * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* aligned = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>(aligned);
@@ -611,24 +596,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &sm.abort_flag;
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 4);
-      mbar_init(&sm.p_full[i], 4);
-      mbar_init(&sm.o_full[i], 1);
+      mbar_init(&sm.p_full[i], 8);
+      mbar_init(&sm.pv_done[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.route_full[i], 1);
       mbar_init(&sm.route_empty[i], 12);  // 2 producers + 2 MMA issuers + 8 softmax warps
       mbar_init(&sm.rfull[i], 1);
     }
-    mbar_init(&sm.o_free, 4);
-    mbar_init(&sm.b_done, 4);
-    mbar_init(&sm.q_free, 2);  // one commit per MMA issuer
+    mbar_init(&sm.o_free[0], 8);
+    mbar_init(&sm.o_free[1], 8);
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_free, 1);
     mbar_init(&sm.mma_done[0], 1);
     mbar_init(&sm.mma_done[1], 1);
     sm.abort_flag = 0;
@@ -639,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 12 && lane == 0) {
+    prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
@@ -646,18 +636,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp >= 12) {
-    regs_dec<kRegsIssue>();
-  } else if (warp >= 8) {
-    regs_dec<kRegsRouting>();
-  } else {
-    regs_inc<kRegsSoftmax>();
-  }
 
   if (warp >= 8 && warp < 12) {
     // ======================= routing =======================
     const int rt = tid - 256;
     uint32_t chunk_ctr = 0;  // routing chunks consumed so far (buffer parity)
+    uint32_t q_loads = 0;    // Q tiles requested so far (q_full phase)
     for (int n = 0;; ++n) {
       const int s = n & 1;
       if (n >= 2) {
@@ -688,30 +672,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.cmax[s][0] = sm.cmax[s][1] = -INFINITY;
         }
       }
-      uint32_t qw[D / 2];
-      load_q_rows<D>(P, bh, pair, rt, qw);
-      if (n >= 1) {  // the Q slot is free once every QK of the previous unit has completed
-        const bool okq = mbar_wait(&sm.q_free, (n - 1) & 1, abort_flag, st, kSiteQFree, u);
-        if (named_bar_or(1, 128, !okq)) break;
-      }
-      tc_fence_after();
-      store_q_tmem<D>(tmem, rt, qw);
-      tc_fence_before();
       named_bar_sync(1, 128);
+      // the list is complete: producers may run ahead into this unit
       if (rt == 0) {
         sm.unit[s] = u;
         mbar_arrive(&sm.route_full[s]);
         SOLATTN_TRACE_EVENT(14, n);
       }
+      // the Q tile is free once every QK of the previous unit has completed
+      bool okq = true;
+      if (rt == 0) {
+        if (n >= 1) okq = mbar_wait(&sm.q_free, (n - 1) & 1, abort_flag, st, kSiteQFree, u);
+        if (okq) {
+          ++q_loads;
+          mbar_arrive_expect_tx(&sm.q_full, kBM * D * 2);
+#pragma unroll
+          for (int pnl = 0; pnl < D / 64; ++pnl)
+            tma_load_3d(&sm.qt[pnl * kBM * 128], &tmQ, &sm.q_full, pnl * 64, pair * kBM, bh);
+        }
+      }
+      if (named_bar_or(1, 128, !okq)) break;
     }
+    if (rt == 0 && q_loads > 0) mbar_wait_quiet(&sm.q_full, (q_loads - 1) & 1);  // teardown: the last Q copy landed
   } else if (warp == 12 || warp == 14) {
-    // ======================= TMA producers: warp 12 = K tiles, warp 14 = V tiles =======================
+    // ======================= TMA producers: warp 12 = K tiles, warp 14 = V blocks =======================
     const bool isK = warp == 12;
-    uint64_t* full = isK ? sm.k_full : sm.v_full;
-    uint64_t* empty = isK ? sm.k_empty : sm.v_empty;
-    const CUtensorMap* map = isK ? &tmK : &tmV;
-    uint8_t* ring = isK ? &sm.kt[0][0] : &sm.vt[0][0];
-    uint32_t g = 0;
+    uint32_t g = 0;  // K: global tile index; V: global block index
     for (int n = 0;; ++n) {
       const int s = n & 1;
       if (!warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullProd, 0)) break;
@@ -719,63 +705,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u < 0) break;
       const int T = sm.count[s];
       const int bh = u / P.npairs;
-      int t = 0;
-      for (; t < T; ++t) {
-        const int j = ROUTE ? (sm.list[s][t] & 0x3FFF) : t;
-        const uint32_t gt = g + t, stg = gt % kStages, r = gt / kStages;
-        if (r >= 1 && !warp_wait(&empty[stg], (r - 1) & 1, abort_flag, st, isK ? kSiteKEmpty : kSiteVEmpty, u)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(&full[stg], kBN * D * 2);
+      bool ok = true;
+      KeyWalk<ROUTE> walk(sm.bits[s][0], sm.bits[s][1]);
+      if (isK) {
+        const int TT = (T + 1) / 2;
+        int t = 0;
+        for (; t < TT; ++t) {
+          const uint32_t gt = g + t, stg = gt % KS, r = gt / KS;
+          if (r >= 1 && !warp_wait(&sm.k_empty[stg], (r - 1) & 1, abort_flag, st, kSiteKEmpty, u)) break;
+          const int nb = (2 * t + 1 < T) ? 2 : 1;
+          int jj[2];
+          jj[0] = walk.next() & 0x3FFF;
+          jj[1] = nb == 2 ? (walk.next() & 0x3FFF) : 0;
+          if (elect_one()) {
+            SOLATTN_TRACE_EVENT(15, gt);
+            mbar_arrive_expect_tx(&sm.k_full[stg], nb * kBN * D * 2);
+            for (int h = 0; h < nb; ++h) {
 #pragma unroll
-          for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(ring + stg * (kBN * D * 2) + pnl * 8192, map, &full[stg], pnl * 64, j * kBN, bh);
+              for (int pnl = 0; pnl < D / 64; ++pnl)
+                tma_load_3d(&sm.kt[stg][pnl * kBM * 128 + h * kBN * 128], &tmK, &sm.k_full[stg], pnl * 64,
+                            jj[h] * kBN, bh);
+            }
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        g += t;
+        ok = t == TT;
+      } else {
+        int t = 0;
+        for (; t < T; ++t) {
+          const int j = walk.next() & 0x3FFF;
+          const uint32_t gt = g + t, stg = gt % VS, r = gt / VS;
+          if (r >= 1 && !warp_wait(&sm.v_empty[stg], (r - 1) & 1, abort_flag, st, kSiteVEmpty, u)) break;
+          if (elect_one()) {
+            SOLATTN_TRACE_EVENT(16, gt);
+            mbar_arrive_expect_tx(&sm.v_full[stg], kBN * D * 2);
+#pragma unroll
+            for (int pnl = 0; pnl < D / 64; ++pnl)
+              tma_load_3d(&sm.vt[stg][pnl * kBN * 128], &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh);
+          }
+          __syncwarp();
+        }
+        g += t;
+        ok = t == T;
       }
-      g += t;
-      if (t < T) break;  // aborted
+      if (!ok) break;  // aborted
       if (elect_one()) mbar_arrive(&sm.route_empty[s]);
       __syncwarp();
     }
     if (lane == 0) {  // teardown: every issued copy lands before the CTA exits
-      const uint32_t first = g > static_cast<uint32_t>(kStages) ? g - kStages : 0u;
-      for (uint32_t gt = first; gt < g; ++gt) mbar_wait_quiet(&full[gt % kStages], (gt / kStages) & 1);
+      const uint32_t depth = isK ? KS : VS;
+      const uint32_t first = g > depth ? g - depth : 0u;
+      for (uint32_t gt = first; gt < g; ++gt) {
+        if (isK) mbar_wait_quiet(&sm.k_full[gt % KS], (gt / KS) & 1);
+        else mbar_wait_quiet(&sm.v_full[gt % VS], (gt / VS) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == 13 || warp == 15) {
-    // ======================= MMA issuers: warp 13 for group A, warp 15 for group B =======================
-    // For the group's own tiles t (global tile parity = group): QK of the next
-    // own tile as soon as the group has read the S of the current one (one S
-    // buffer per group), then PV of the current one once its P is stored.
-    // Waits sleep on their mbarrier (bounded); one lane issues.
-    const int grp = warp == 13 ? 0 : 1;
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+    // ======================= MMA issuers: warp 13 = QK, warp 15 = PV =======================
+    // QK(t) goes into S slot t % 3 as soon as its K tile has landed and the
+    // PV that last read P from that slot (tile t - 3) has completed: MMAs into
+    // different accumulators are not ordered with each other, so the slot is
+    // reused only after pv_done (waited once per tile, in order). The S ring
+    // therefore runs up to two tiles ahead of the softmax. PV(t) goes as soon
+    // as all eight softmax warps have stored P(t) and its V blocks have landed.
+    const bool isQK = warp == 13;
+    constexpr uint32_t idesc_qk2 = idesc_bf16_f32(kBM, 2 * kBN, false, false);
+    constexpr uint32_t idesc_qk1 = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-    constexpr uint32_t kTileBytes = kBN * D * 2;
+    const uint64_t qdesc = sw128_desc(smem_u32(&sm.qt[0]), 16, 1024);
     const uint64_t kdesc0 = sw128_desc(smem_u32(&sm.kt[0][0]), 16, 1024);
     const uint64_t vdesc0 = sw128_desc(smem_u32(&sm.vt[0][0]), 8192, 1024);
-    const uint32_t colS = tmem + kColS + grp * 64, colP = tmem + kColP + grp * 32, colO = tmem + kColO + grp * 128;
-    uint32_t g = 0;
+    const uint32_t colO = tmem + kColO;
+    uint32_t gtile = 0, gblk = 0;
+    uint32_t pv_waited = 0;  // QK issuer: tiles whose PV completion it has observed
     bool ok = true;
-    auto issue_qk = [&](uint32_t gt, int u, bool last) -> bool {
-      const uint32_t stg = gt % kStages, use = gt >> 1;
-      if (use >= 1 && !warp_wait(&sm.s_free[grp], (use - 1) & 1, abort_flag, st, kSiteSFree, u)) return false;
-      if (!warp_wait(&sm.k_full[stg], (gt / kStages) & 1, abort_flag, st, kSiteKFull, u)) return false;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t kd = kdesc0 + ((stg * kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ts(colS, tmem + kColQ + kk * 8, kd + ((((kk / 4) * 8192) + (kk % 4) * 32) >> 4), idesc_qk,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(&sm.s_full[grp]);
-        mma_commit(&sm.k_empty[stg]);
-        if (last) mma_commit(&sm.q_free);
-        SOLATTN_TRACE_EVENT(10, gt);
-      }
-      __syncwarp();
-      return true;
-    };
     for (int n = 0; ok; ++n) {
       const int s = n & 1;
       if (!warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullMma, 0)) break;
@@ -783,28 +788,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      const int t0 = ((g & 1u) == static_cast<uint32_t>(grp)) ? 0 : 1;  // first own tile of the unit
-      if (t0 >= T) {  // no own tile: still release the Q slot and keep o_free's phase
-        if (elect_one()) mma_commit(&sm.q_free);
-        __syncwarp();
-        if (n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) break;
-      } else {
-        ok = issue_qk(g + t0, u, t0 + 2 >= T);
-        if (ok && n >= 1 && !warp_wait(&sm.o_free, (n - 1) & 1, abort_flag, st, kSiteOFree, u)) ok = false;
-        for (int t = t0; t < T && ok; t += 2) {
-          if (t + 2 < T && !(ok = issue_qk(g + t + 2, u, t + 4 >= T))) break;
-          const uint32_t gp = g + t, stp = gp % kStages, usep = gp >> 1;
-          if (!warp_wait(&sm.p_full[grp], usep & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
-          if (!warp_wait(&sm.v_full[stp], (gp / kStages) & 1, abort_flag, st, kSiteVFull, u)) { ok = false; break; }
+      const int TT = (T + 1) / 2;
+      if (isQK) {
+        if (!warp_wait(&sm.q_full, n & 1, abort_flag, st, kSiteQFull, u)) break;
+        if (TT == 0) {  // nothing to multiply: release the Q tile
+          if (elect_one()) mma_commit(&sm.q_free);
+          __syncwarp();
+        }
+        for (int t = 0; t < TT && ok; ++t) {
+          const uint32_t gt = gtile + t, stg = gt % KS, slot = gt % 3;
+          for (; pv_waited + 3 <= gt && ok; ++pv_waited)
+            ok = warp_wait(&sm.pv_done[pv_waited % 3], (pv_waited / 3) & 1, abort_flag, st, kSitePvDone, u);
+          if (ok) ok = warp_wait(&sm.k_full[stg], (gt / KS) & 1, abort_flag, st, kSiteKFull, u);
+          if (!ok) break;
+          if (lane == 0) SOLATTN_TRACE_EVENT(17, gt);
           tc_fence_after();
           if (elect_one()) {
-            SOLATTN_TRACE_EVENT(11, gp);
-            const uint64_t vd = vdesc0 + ((stp * kTileBytes) >> 4);
+            const uint64_t kd = kdesc0 + ((stg * (kBM * D * 2)) >> 4);
+            const uint32_t idesc = (2 * t + 1 < T) ? idesc_qk2 : idesc_qk1;
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              mma_ts(colO, colP + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (t > t0 || kk > 0) ? 1u : 0u);
-            mma_commit(&sm.v_empty[stp]);
-            mma_commit(&sm.o_full[grp]);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (((kk / 4) * kBM * 128) + (kk % 4) * 32) >> 4;
+              mma_ss(tmem + slot * 128, qdesc + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.s_full[slot]);
+            mma_commit(&sm.k_empty[stg]);
+            if (t == TT - 1) mma_commit(&sm.q_free);
+            SOLATTN_TRACE_EVENT(10, gt);
+          }
+          __syncwarp();
+        }
+      } else {
+        // O is free once the epilogue has read the previous unit's
+        if (n >= 1 && !warp_wait(&sm.o_free[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, st, kSiteOFree, u)) break;
+        for (int t = 0; t < TT && ok; ++t) {
+          const uint32_t gt = gtile + t;
+          const int nb = (2 * t + 1 < T) ? 2 : 1;
+          if (!warp_wait(&sm.p_full[gt % 3], (gt / 3) & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
+          if (lane == 0) SOLATTN_TRACE_EVENT(12, gt);
+          uint32_t stv[2];
+          for (int h = 0; h < nb && ok; ++h) {
+            const uint32_t gv = gblk + 2 * t + h;
+            stv[h] = gv % VS;
+            ok = warp_wait(&sm.v_full[stv[h]], (gv / VS) & 1, abort_flag, st, kSiteVFull, u);
+          }
+          if (!ok) break;
+          if (lane == 0) SOLATTN_TRACE_EVENT(18, gt);
+          tc_fence_after();
+          if (elect_one()) {
+            SOLATTN_TRACE_EVENT(11, gt);
+            const uint32_t colP = tmem + (gt % 3) * 128;
+            for (int h = 0; h < nb; ++h) {
+              const uint64_t vd = vdesc0 + ((stv[h] * (kBN * D * 2)) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ts(colO, colP + h * 32 + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                       (t > 0 || h > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(&sm.v_empty[stv[h]]);
+            }
+            mma_commit(&sm.pv_done[gt % 3]);
           }
           __syncwarp();
         }
@@ -812,148 +854,156 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (elect_one()) mma_commit(&sm.route_empty[s]);
       __syncwarp();
-      g += T;
+      gtile += TT;
+      gblk += T;
     }
-    if (elect_one()) mma_commit(&sm.mma_done[grp]);  // teardown: issued MMAs complete before TMEM is freed
+    const int me = isQK ? 0 : 1;
+    if (elect_one()) mma_commit(&sm.mma_done[me]);  // teardown: issued MMAs complete before TMEM is freed
     __syncwarp();
-    mbar_wait_quiet(&sm.mma_done[grp], 0);
+    mbar_wait_quiet(&sm.mma_done[me], 0);
     __syncwarp();
-  } else {
-    // ======================= softmax groups A (warps 0-3) and B (4-7) =======================
-    const int grp = warp >> 2;   // 0 = A (even global tiles), 1 = B (odd)
-    const int r = tid & 127;     // row of the unit == TMEM lane
-    const int blk = r >> 6;      // which of the two query blocks
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  } else if (warp < 8) {
+    // ======================= softmax =======================
+    const int q4 = warp & 3, hh = warp >> 2;  // row group, key half of the tile
+    const int r = q4 * 32 + lane;             // row of the unit == TMEM lane
+    const int blk = r >> 6;                   // which of the two query blocks (warp-uniform)
+    const int pb = 2 + q4;                    // named barrier of warps q4 and q4 + 4 (same rows)
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const float sl2 = kLog2e * rsqrtf(static_cast<float>(D));
     const int nlast = P.N - (P.NB - 1) * kBN;
-    const uint32_t colS = tmem + kColS + grp * 64 + lane_off;
-    const uint32_t colP = tmem + kColP + grp * 32 + lane_off;
-    const uint32_t colO = tmem + kColO + grp * 128 + lane_off;
-    uint32_t g = 0;
+    constexpr int DH = D / 2;                 // O / output columns owned by this warp
+    const uint32_t colO = tmem + kColO + lane_off + hh * DH;
+    uint32_t gtile = 0;
     for (int n = 0;; ++n) {
       const int s = n & 1;
-      if (!warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullSoft, 0)) break;
+      bool okr = warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullSoft, 0);
+      if (named_bar_or(pb, 64, !okr)) break;
       tc_fence_after();
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      const int bh = u / P.npairs, pair = u % P.npairs;
-      float m = -INFINITY, l = 0.f;
-      bool ok = true, first = true;
-      uint32_t last_use = 0;
-      for (int t = ((g & 1u) == static_cast<uint32_t>(grp)) ? 0 : 1; t < T; t += 2) {
-        const uint32_t gt = g + t, use = gt >> 1;
-        const uint32_t entry = ROUTE ? sm.list[s][t] : (static_cast<uint32_t>(t) | 0xC000u);
-        const int j = entry & 0x3FFF;
-        const bool mine = (entry >> (14 + blk)) & 1u;  // warp-uniform
-        if (!warp_wait(&sm.s_full[grp], use & 1, abort_flag, st, kSiteSFull, u)) { ok = false; break; }
-        tc_fence_after();
-        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 0, gt);
-        uint32_t sv[32], sw[32];
-        if (mine) {
-          tmem_ld32(colS, sv);
-          tmem_ld32(colS + 32, sw);
-          tmem_wait_ld();
+      const int TT = (T + 1) / 2;
+      float m = -INFINITY, l = 0.f;  // m: the row's shared reference max; l: this half's sum
+      bool ok = true;
+      KeyWalk<ROUTE> walk(sm.bits[s][0], sm.bits[s][1]);
+      for (int t = 0; t < TT; ++t) {
+        const uint32_t gt = gtile + t, slot = gt % 3;
+        const uint32_t colS = tmem + slot * 128 + lane_off;
+        const int nb = (2 * t + 1 < T) ? 2 : 1;
+        uint32_t entry = 0u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t e = h < nb ? walk.next() : 0u;
+          if (h == hh) entry = e;
         }
+        const bool kept = (entry >> (14 + blk)) & 1u;
+        const int nv = ((entry & 0x3FFF) == static_cast<uint32_t>(P.NB - 1)) ? nlast : kBN;
+        const bool okw = warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
+        tc_fence_after();
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(0, gt);
+        uint32_t sv[64];
+        if (kept && okw) tmem_ld32x2_wait(colS + 64 * hh, colS + 64 * hh + 32, sv);
+        const float mx = (kept && okw) ? tile_max(sv, nv) * sl2 : -INFINITY;
+        // Does a row of this group need a new reference max (or did a wait fail)?
+        // The barrier also orders this group's S reads before the other half's
+        // P stores into the same columns.
         tc_fence_before();
-        __syncwarp();
-        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 1, gt);
-        if (lane == 0) mbar_arrive(&sm.s_free[grp]);
-        float rescale = 1.f;
-        bool need = false;
-        uint32_t pw[32];
-        if (mine) {
-          need = softmax_max(sv, sw, (j == P.NB - 1) ? nlast : kBN, sl2, m, rescale);
-          if (need) l *= rescale;
-          if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 2, gt);
-          const uint64_t sc2 = f2_dup(sl2);
-          const uint64_t nm2 = f2_dup(-m);
-          softmax_slice(&sv[0], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[0]));
-          softmax_slice(&sv[16], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[8]));
-          softmax_slice(&sw[0], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[16]));
-          softmax_slice(&sw[16], sc2, nm2, l, *reinterpret_cast<uint32_t(*)[8]>(&pw[24]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pw[c] = 0u;
-        }
-        // this group's previous PV must be complete: it read the P buffer and wrote O
-        if (!first && !warp_wait(&sm.o_full[grp], (use - 1) & 1, abort_flag, st, kSiteOFull, u)) { ok = false; break; }
+        const bool any = named_bar_or(pb, 64, !okw || mx > m + kRescaleSlack);
         tc_fence_after();
-        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 3, gt);
-        if (__any_sync(0xffffffffu, need)) {
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(1, gt);
+        if (any) {
+          sm.xm[r][hh] = okw ? mx : NAN;
+          named_bar_sync(pb, 64);
+          const float mo = sm.xm[r][hh ^ 1];
+          if (__any_sync(0xffffffffu, !okw || mo != mo)) { ok = false; break; }  // identical in both warps
+          const float mrow = fmaxf(mx, mo);
+          float rescale = 1.f;
+          bool need = false;
+          if (mrow > m + kRescaleSlack) {
+            need = m != -INFINITY;
+            if (need) rescale = ex2_approx(m - mrow);
+            m = mrow;
+          }
+          if (__any_sync(0xffffffffu, need)) {
+            // O must hold every PV up to the previous tile before it is rescaled
+            const uint32_t gp = gt - 1;
+            const bool okp = warp_wait(&sm.pv_done[gp % 3], (gp / 3) & 1, abort_flag, st, kSitePvDone, u);
+            if (named_bar_or(pb, 64, !okp)) { ok = false; break; }
+            tc_fence_after();
+            l *= rescale;
+#pragma unroll 1
+            for (int ch = 0; ch < DH / 16; ++ch) {
+              uint32_t ov[16];
+              tmem_ld16_wait(colO + ch * 16, ov);
 #pragma unroll
-          for (int ch = 0; ch < D / 16; ++ch) {
-            uint32_t ov[16];
-            tmem_ld16(colO + ch * 16, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * rescale);
-            tmem_st16(colO + ch * 16, ov);
+              for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * rescale);
+              tmem_st16_wait(colO + ch * 16, ov);
+            }
           }
         }
-        tmem_st32(colP, pw);
-        tmem_wait_st();
+        // ---- P = 2^(S sl2 - m) in bf16 for this key half, over S's first 64 columns
+        if (hh < nb) {
+          uint32_t pw[32];
+          if (kept) {
+            const uint64_t sc2 = f2_dup(sl2);
+            const uint64_t nm2 = f2_dup(-m);
+            uint64_t lsum = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              softmax_slice(&sv[16 * q], sc2, nm2, lsum, *reinterpret_cast<uint32_t(*)[8]>(&pw[8 * q]));
+            float l0, l1;
+            f2_split(lsum, l0, l1);
+            l += l0 + l1;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pw[c] = 0u;
+          }
+          tmem_st32_wait(colS + 32 * hh, pw);
+        }
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(3, gt);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[grp]);
-        if ((tid & 127) == 0) SOLATTN_TRACE_EVENT(grp * 5 + 4, gt);
-        first = false;
-        last_use = use;
+        if (lane == 0) mbar_arrive(&sm.p_full[slot]);
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(4, gt);
       }
       if (!ok) break;
-      // this group's last PV of the unit
-      if (!first) {
-        if (!warp_wait(&sm.o_full[grp], last_use & 1, abort_flag, st, kSiteOFull, u)) break;
-        tc_fence_after();
+      // ---------------- epilogue: O and l merged with the correction ----------------
+      const int bh = u / P.npairs, pair = u % P.npairs;
+      const bool hasO = TT > 0;
+      bool oke = true;
+      if (hasO) {  // the unit's last PV has completed
+        const uint32_t gl = gtile + TT - 1;
+        oke = warp_wait(&sm.pv_done[gl % 3], (gl / 3) & 1, abort_flag, st, kSitePvDone, u);
       }
-      if (grp == 1) {
-        sm.mB[s][r] = m;
-        sm.lB[s][r] = l;
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sm.b_done);
-          mbar_arrive(&sm.route_empty[s]);
-        }
-        g += T;
-        continue;
-      }
-      // ---------------- epilogue (group A): merge A, B and the correction ----------------
-      if (!warp_wait(&sm.b_done, n & 1, abort_flag, st, kSiteBDone, u)) break;
-      const bool hasA = !first;
-      const int tilesB = ((g & 1u) == 1u) ? (T + 1) / 2 : T / 2;
-      const bool hasB = tilesB > 0;
-      const float mB = sm.mB[s][r], lB = sm.lB[s][r];
+      sm.xl[r][hh] = l;
+      if (named_bar_or(pb, 64, !oke)) break;
+      tc_fence_after();
+      const float lrow = sm.xl[r][0] + sm.xl[r][1];
+      named_bar_sync(pb, 64);  // both halves have read xl
       const float mc = sm.cmax[s][blk] * kLog2e;
       const float cd = sm.cden[s][blk];
-      const float mf = fmax3(m, mB, mc);
+      const float mf = fmaxf(m, mc);
       const float wa = (m == -INFINITY) ? 0.f : ex2_approx(m - mf);
-      const float wb = (mB == -INFINITY) ? 0.f : ex2_approx(mB - mf);
       const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - mf);
-      const float L = fmaf(l, wa, fmaf(lB, wb, cd * wc));
+      const float L = fmaf(lrow, wa, cd * wc);
       const float inv = 1.f / L;
       const int row = pair * kBM + r;
       const bool valid = row < P.N;
-      uint16_t* orow = P.out + (static_cast<long long>(bh) * P.N + row) * D;
-      for (int ch = 0; ch < D / 16; ++ch) {
+      uint16_t* orow = P.out + (static_cast<long long>(bh) * P.N + row) * D + hh * DH;
+#pragma unroll 1
+      for (int ch = 0; ch < DH / 16; ++ch) {
         float y[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) y[e] = 0.f;
         if constexpr (ROUTE) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) y[e] = sm.cnum[s][blk][ch * 16 + e] * wc;
+          for (int e = 0; e < 16; ++e) y[e] = sm.cnum[s][blk][hh * DH + ch * 16 + e] * wc;
         }
-        uint32_t o[16];
-        if (hasA) {
-          tmem_ld16(colO + ch * 16, o);
-          tmem_wait_ld();
+        if (hasO) {
+          uint32_t o[16];
+          tmem_ld16_wait(colO + ch * 16, o);
 #pragma unroll
           for (int e = 0; e < 16; ++e) y[e] = fmaf(__uint_as_float(o[e]), wa, y[e]);
-        }
-        if (hasB) {
-          tmem_ld16(colO + 128 + ch * 16, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) y[e] = fmaf(__uint_as_float(o[e]), wb, y[e]);
         }
         if (valid) {
           uint32_t pk[8];
@@ -964,14 +1014,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (valid && P.lse) P.lse[static_cast<long long>(bh) * P.N + row] = (mf + __log2f(L)) * kLn2;
+      if (valid && P.lse && hh == 0) P.lse[static_cast<long long>(bh) * P.N + row] = (mf + __log2f(L)) * kLn2;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sm.o_free);
+        mbar_arrive(&sm.o_free[s]);
         mbar_arrive(&sm.route_empty[s]);
       }
-      g += T;
+      gtile += TT;
     }
   }
 
@@ -1002,14 +1052,14 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH][N][D] bf16 viewed as a 3D tensor (D fastest); box = 64 columns x 64 rows,
-// 128-byte swizzle; rows past N read as zero.
-bool make_kv_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+// [BH][N][D] bf16 viewed as a 3D tensor (D fastest); box = 64 columns x `rows`
+// rows, 128-byte swizzle; rows past N read as zero.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBN), 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1018,8 +1068,9 @@ bool make_kv_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
 
 template <int D, bool ROUTE>
 cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
-  CUtensorMap tmK, tmV;
-  if (!make_kv_map(&tmK, a.k, a.BH, a.N, D) || !make_kv_map(&tmV, a.v, a.BH, a.N, D))
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_map(&tmQ, a.q, a.BH, a.N, D, kBM) || !make_map(&tmK, a.k, a.BH, a.N, D, kBN) ||
+      !make_map(&tmV, a.v, a.BH, a.N, D, kBN))
     return cudaErrorInvalidValue;
   Params p{};
   p.q = a.q;
@@ -1043,7 +1094,7 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.units < num_sms ? p.units : num_sms;
-  solattn_fwd_kernel<D, ROUTE><<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
+  solattn_fwd_kernel<D, ROUTE><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
