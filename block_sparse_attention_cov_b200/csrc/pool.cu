@@ -122,7 +122,7 @@ constexpr int kRows = 32;   // key blocks staged per trip
 template <int D>
 struct KeyStatsSmem {
   float part[D][D];         // this CTA's sum of deviation outer products
-  float dev[kRows][D];      // staged deviations
+  float dev[2][kRows][D];   // staged deviations, double-buffered
   float colpart[256 / (D / 4)][D];
   float csum[D];            // this CTA's column sums (read by the whole cluster)
   float mean[D];
@@ -183,24 +183,39 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(256)
   for (int x = 0; x < TT; ++x)
 #pragma unroll
     for (int y = 0; y < TT; ++y) acc[x][y] = 0.f;
-  for (int c0 = j0; c0 < j1; c0 += kRows) {
+  // staged through registers: the next 32 key blocks are in flight while the
+  // current ones are multiplied
+  constexpr int PER = kRows * D / 4 / 256;  // float4 per thread per stage
+  float4 pre[PER];
+  auto fetch = [&](int c0) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = tid + 256 * i, r = e / (D / 4), c = (e % (D / 4)) * 4;
+      pre[i] = (c0 + r < j1) ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(c0 + r) * D + c))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  if (j0 < j1) fetch(j0);
+  for (int c0 = j0, it = 0; c0 < j1; c0 += kRows, ++it) {
     const int nr = min(kRows, j1 - c0);
-    for (int e = tid; e < kRows * D / 4; e += 256) {
-      const int r = e / (D / 4), c = (e % (D / 4)) * 4;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    float (*dv)[D] = sm.dev[it & 1];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = tid + 256 * i, r = e / (D / 4), c = (e % (D / 4)) * 4;
+      float4 x = pre[i];
       if (r < nr) {
-        x = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(c0 + r) * D + c));
         x.x -= sm.mean[c]; x.y -= sm.mean[c + 1]; x.z -= sm.mean[c + 2]; x.w -= sm.mean[c + 3];
       }
-      *reinterpret_cast<float4*>(&sm.dev[r][c]) = x;
+      *reinterpret_cast<float4*>(&dv[r][c]) = x;  // rows past the slice stay zero
     }
     __syncthreads();
+    if (c0 + kRows < j1) fetch(c0 + kRows);
     for (int r = 0; r < nr; ++r) {
       float av[TT], bv[TT];
 #pragma unroll
       for (int h = 0; h < TT / 4; ++h) {
-        const float4 x = *reinterpret_cast<const float4*>(&sm.dev[r][64 * h + 4 * ta]);
-        const float4 y = *reinterpret_cast<const float4*>(&sm.dev[r][64 * h + 4 * tb]);
+        const float4 x = *reinterpret_cast<const float4*>(&dv[r][64 * h + 4 * ta]);
+        const float4 y = *reinterpret_cast<const float4*>(&dv[r][64 * h + 4 * tb]);
         av[4 * h] = x.x; av[4 * h + 1] = x.y; av[4 * h + 2] = x.z; av[4 * h + 3] = x.w;
         bv[4 * h] = y.x; bv[4 * h + 1] = y.y; bv[4 * h + 2] = y.z; bv[4 * h + 3] = y.w;
       }
@@ -209,7 +224,6 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(256)
 #pragma unroll
         for (int y = 0; y < TT; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
-    __syncthreads();
   }
 #pragma unroll
   for (int x = 0; x < TT; ++x) {
