@@ -190,6 +190,72 @@ def route(q: np.ndarray, k: np.ndarray, beta: float) -> dict:
 
 
 # --------------------------------------------------------------------------
+# Other kept-set rules (ablation) and always-kept prefix blocks
+# --------------------------------------------------------------------------
+# The pages compare the per-row threshold with the top-k and top-p selections
+# of earlier methods (paithon.it, "Una soglia per ogni riga": a global top-k
+# or top-p gives every row the same budget or needs a sort; "I numeri":
+# routing-time comparison threshold / top-k / top-p) and keep text tokens of
+# joint attention always exact ("Dove leggere con attenzione"). They define
+# neither rule; the readings used here:
+#  * top-k keeps the blocks whose proxy score is at least the k-th largest of
+#    the row (k clamped to [0, N_b]; equal scores at the cut are all kept);
+#  * top-p keeps the blocks whose proxy score is at least v*, the largest
+#    value whose superlevel set carries a fraction >= p of the row's mass
+#    sum_j n_j exp(s_hat_ij) (the weight a skipped block would get); p <= 0
+#    keeps nothing, p >= 1 keeps everything;
+#  * forced blocks 0 .. n_forced - 1 are kept in every row in addition to the
+#    rule's set.
+def topk_mask(shat: np.ndarray, k: int) -> np.ndarray:
+    """[N_b, N_b] bool: s_hat_ij >= the k-th largest value of row i."""
+    nb = shat.shape[1]
+    if k <= 0:
+        return np.zeros(shat.shape, bool)
+    if k >= nb:
+        return np.ones(shat.shape, bool)
+    kth = -np.sort(-shat, axis=1)[:, k - 1]
+    return shat >= kth[:, None]
+
+
+def topp_mask(shat: np.ndarray, counts: np.ndarray, p: float) -> np.ndarray:
+    """[N_b, N_b] bool: s_hat_ij >= v*_i, v*_i the largest score whose
+    superlevel set holds >= p of sum_j n_j exp(s_hat_ij)."""
+    nb = shat.shape[1]
+    if p <= 0.0:
+        return np.zeros(shat.shape, bool)
+    if p >= 1.0:
+        return np.ones(shat.shape, bool)
+    mask = np.zeros(shat.shape, bool)
+    for i in range(shat.shape[0]):
+        order = np.argsort(-shat[i], kind="stable")
+        w = counts[order] * np.exp(shat[i, order] - shat[i, order[0]])
+        cum = np.cumsum(w)
+        kp = int(np.searchsorted(cum, p * cum[-1], side="left"))  # first index with cum >= p * total
+        vstar = shat[i, order[min(kp, nb - 1)]]
+        mask[i] = shat[i] >= vstar
+    return mask
+
+
+def route_rule(q: np.ndarray, k: np.ndarray, rule: str, param: float, n_forced: int = 0) -> dict:
+    """route() with another kept-set rule: rule = "threshold" (param = beta),
+    "topk" (param = k) or "topp" (param = p), plus n_forced always-kept blocks."""
+    r = route(q, k, param if rule == "threshold" else 0.0)
+    if rule == "topk":
+        mask = topk_mask(r["shat"], int(param))
+    elif rule == "topp":
+        mask = topp_mask(r["shat"], block_counts(q.shape[0]).astype(np.float64), float(param))
+    elif rule == "threshold":
+        mask = r["mask"].copy()
+    else:
+        raise ValueError(rule)
+    if n_forced > 0:
+        mask[:, :n_forced] = True
+    r["mask"] = mask
+    r["density"] = mask.sum(axis=1).astype(np.int64)
+    return r
+
+
+# --------------------------------------------------------------------------
 # Step 6: attention with exact kept blocks and zeroth-order correction
 # --------------------------------------------------------------------------
 def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None):

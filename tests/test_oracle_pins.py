@@ -355,3 +355,110 @@ def test_bf16_inputs_pass_through_exactly():
     a = orc._as64(x)
     assert a.dtype == np.float64
     assert np.array_equal(a, x.double().numpy())
+
+
+# ---------------------------------------------------------------------------
+# Other kept-set rules (top-k, top-p) and always-kept prefix blocks: the
+# pages compare the threshold with top-k / top-p routing ("Una soglia per ogni
+# riga", "I numeri") and keep text tokens of joint attention exact ("Dove
+# leggere con attenzione"); the readings are stated in the oracle.
+# ---------------------------------------------------------------------------
+def _proxy(seed, N, d):
+    rng = _rng(seed)
+    q, k = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    qb = np.stack([q[a:b].mean(0) for a, b in orc.block_bounds(N)])
+    kb = np.stack([k[a:b].mean(0) for a, b in orc.block_bounds(N)])
+    return q, k, (qb @ kb.T) / math.sqrt(d)
+
+
+@pytest.mark.parametrize("kk", [0, 1, 3, 7, 10, 25])
+def test_topk_keeps_exactly_the_k_largest(kk):
+    q, k, shat = _proxy(31, 64 * 9 + 17, 32)
+    nb = shat.shape[1]
+    r = orc.route_rule(q, k, "topk", kk)
+    want = min(max(kk, 0), nb)
+    assert (r["density"] == want).all()
+    for i in range(nb):
+        kept, skip = shat[i][r["mask"][i]], shat[i][~r["mask"][i]]
+        if len(kept) and len(skip):
+            assert kept.min() > skip.max()
+        # the kept set is the k largest of the row, found by a full sort
+        assert set(np.nonzero(r["mask"][i])[0]) == set(np.argsort(-shat[i])[:want])
+
+
+def test_topk_ties_at_the_cut_are_all_kept():
+    shat = np.array([[3.0, 1.0, 2.0, 2.0, 0.0]])
+    assert orc.topk_mask(shat, 2).tolist() == [[True, False, True, True, False]]
+    assert orc.topk_mask(shat, 3).tolist() == [[True, False, True, True, False]]
+    assert orc.topk_mask(shat, 4).tolist() == [[True, True, True, True, False]]
+
+
+@pytest.mark.parametrize("p", [0.0, 0.1, 0.5, 0.9, 0.999, 1.0])
+def test_topp_against_brute_force_over_every_cut(p):
+    """Every distinct score is tried as the cut: v* is the largest one whose
+    superlevel set holds >= p of sum_j n_j e^{s_hat_ij} (n_j: valid tokens)."""
+    N = 64 * 7 + 9   # the last block holds 9 tokens: its weight matters
+    q, k, shat = _proxy(32, N, 32)
+    n = np.array([b - a for a, b in orc.block_bounds(N)], dtype=np.float64)
+    r = orc.route_rule(q, k, "topp", p)
+    for i in range(shat.shape[0]):
+        w = n * np.exp(shat[i])
+        total = w.sum()
+        if p <= 0:
+            want = np.zeros(len(w), bool)
+        elif p >= 1:
+            want = np.ones(len(w), bool)
+        else:
+            good = [v for v in shat[i] if w[shat[i] >= v].sum() >= p * total]
+            want = shat[i] >= max(good)
+        assert (r["mask"][i] == want).all(), (i, p)
+
+
+def test_topp_density_is_monotone_in_p():
+    q, k, _ = _proxy(33, 64 * 12, 32)
+    prev = None
+    for p in (0.0, 0.05, 0.2, 0.4, 0.6, 0.8, 0.95, 1.0):
+        d = orc.route_rule(q, k, "topp", p)["density"]
+        if prev is not None:
+            assert (d >= prev).all()
+        prev = d
+    assert (prev == 12).all()
+
+
+def test_forced_blocks_are_kept_and_reproduce_dense_when_all_forced():
+    rng = _rng(34)
+    N, d = 64 * 5 + 30, 32
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    r = orc.route_rule(q, k, "threshold", math.inf, n_forced=2)
+    assert (r["density"] == 2).all() and r["mask"][:, :2].all() and not r["mask"][:, 2:].any()
+    r = orc.route_rule(q, k, "threshold", 0.7, n_forced=3)
+    base = orc.route_rule(q, k, "threshold", 0.7)
+    assert (r["mask"] == (base["mask"] | (np.arange(6) < 3)[None, :])).all()
+    full = orc.route_rule(q, k, "threshold", math.inf, n_forced=6)["mask"]
+    out, _, _ = orc.attend(q, k, v, mask=full)
+    np.testing.assert_allclose(out, _sdpa64(q, k, v), rtol=1e-12, atol=1e-13)
+
+
+def test_topk_all_blocks_is_dense_attention():
+    rng = _rng(35)
+    N, d = 64 * 4 + 3, 64
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    m = orc.route_rule(q, k, "topk", 5)["mask"]
+    out, _, dens = orc.attend(q, k, v, mask=m)
+    assert (dens == 5).all()
+    np.testing.assert_allclose(out, _sdpa64(q, k, v), rtol=1e-12, atol=1e-13)
+
+
+def test_planted_mistakes_in_the_other_rules_are_caught(monkeypatch):
+    # top-p mass without the n_j weights: the brute force (which weighs by n_j) fails
+    real_topp = orc.topp_mask
+    monkeypatch.setattr(orc, "topp_mask", lambda shat, counts, p: real_topp(shat, np.ones_like(counts), p))
+    with pytest.raises(AssertionError):
+        for p in (0.1, 0.5, 0.9, 0.999):
+            test_topp_against_brute_force_over_every_cut(p)
+    monkeypatch.undo()
+    # top-k taking the smallest scores
+    monkeypatch.setattr(orc, "topk_mask", lambda shat, k: shat <= np.sort(shat, axis=1)[:, max(k, 1) - 1:max(k, 1)])
+    with pytest.raises(AssertionError):
+        test_topk_keeps_exactly_the_k_largest(3)
+    monkeypatch.undo()
