@@ -144,16 +144,18 @@ def fwd_traffic(heads):
 
 
 # --------------------------------------------------------------------------- helpers
-def kept_flops(stats, dens, beta, N, d):
+def kept_flops(stats, dens, beta, N, d, rule="threshold", n_forced=0):
     """Algorithmic kept-block FLOPs: 4 d n_i sum_{j in S_i} n_j over every (b, h, i).
-    Only the last key block can be partial; whether it is kept by row i is
-    recomputed from the pooled statistics (bookkeeping only)."""
+    Only the last key block can be partial; with the threshold rule whether row
+    i keeps it is recomputed from the pooled statistics (bookkeeping only); with
+    the top-k / top-p rules it is counted as a full block (an overcount below
+    1e-4 of the work at 75.6K tokens)."""
     nb = math.ceil(N / 64)
     n_last = N - 64 * (nb - 1)
     n_i = torch.full((nb,), 64.0, device=dens.device, dtype=torch.float64)
     n_i[-1] = n_last
     cols = 64.0 * dens.double()
-    if n_last < 64:
+    if n_last < 64 and rule == "threshold" and n_forced < nb:
         qbar, kbar = stats.view("qbar").double(), stats.view("kbar").double()
         s = 1.0 / math.sqrt(d)
         sh = s * (qbar @ kbar[..., -1, :].unsqueeze(-1)).squeeze(-1)
@@ -275,13 +277,15 @@ def run_ours(args, rank, world, local_rank):
     nb = math.ceil(N / 64)
     dens = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
 
+    rule_kw = {"rule": args.rule, "topk": args.topk, "topp": args.topp, "n_forced": args.n_forced}
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
         sa.pool(q, k, v, stats)
         if ev is not None:
             ev[1].record(stream)
-        sa.forward(q, k, v, stats, beta, out=out, lse=lse, density=dens, ws=ws)
+        sa.forward(q, k, v, stats, beta, out=out, lse=lse, density=dens, ws=ws, **rule_kw)
         if ev is not None:
             ev[2].record(stream)
 
@@ -290,7 +294,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if sa.status(ws) != 0:
         raise RuntimeError(f"device status {sa.status(ws)} after warm-up")
-    kflops = kept_flops(stats, dens, beta, N, d)
+    kflops = kept_flops(stats, dens, beta, N, d, args.rule, args.n_forced)
     mean_density = float(dens.double().mean().item()) / nb
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -351,7 +355,7 @@ def run_ours(args, rank, world, local_rank):
             kd.copy_(kp, non_blocking=True)
             vd.copy_(vp, non_blocking=True)
             sa.pool(qd, kd, vd, stats)
-            sa.forward(qd, kd, vd, stats, beta, out=out, lse=lse, density=dens, ws=ws)
+            sa.forward(qd, kd, vd, stats, beta, out=out, lse=lse, density=dens, ws=ws, **rule_kw)
             out_h.copy_(out, non_blocking=True)
             lse_h.copy_(lse, non_blocking=True)
             dens_h.copy_(dens, non_blocking=True)
@@ -407,6 +411,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; bf16)",
         "config": {
             "workload": args.workload, "B": B, "H": H, "N": N, "d": d, "grid": list(wl.grid), "beta": beta,
+            "rule": args.rule, **({"topk": args.topk} if args.rule == "topk" else {}),
+            **({"topp": args.topp} if args.rule == "topp" else {}),
+            **({"n_forced": args.n_forced} if args.n_forced else {}),
             "mean_density": mean_density, "global_batch": B * world, "seq_len": N,
             "parallelism": f"heads-independent replicas x{world}",
             "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no explicit flush" % (B * H * N * d * 2 / 1e6),
@@ -453,6 +460,12 @@ def main():
     ap.add_argument("--beta", type=float, default=None)
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--cpu-blocks", type=int, default=600)
+    ap.add_argument("--rule", choices=["threshold", "topk", "topp"], default="threshold",
+                    help="kept-set rule (the method is 'threshold'; top-k / top-p are the ablation rules)")
+    ap.add_argument("--topk", type=int, default=177, help="top-k rule: blocks per query block (15 %% of 1182)")
+    ap.add_argument("--topp", type=float, default=0.1612,
+                    help="top-p rule: mass fraction (0.1612 gives a 15 %% mean density on the Wan-like inputs)")
+    ap.add_argument("--n-forced", type=int, default=0, help="leading key blocks always kept")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-dense", action="store_true")

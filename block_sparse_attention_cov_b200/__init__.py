@@ -106,9 +106,17 @@ def workspace(device=None) -> torch.Tensor:
     return torch.empty(_lib.WORKSPACE_BYTES, dtype=torch.uint8, device=device or "cuda")
 
 
-def forward(q, k, v, stats: PooledStats, beta: float, out=None, lse=None, density=None, ws=None,
-            want_lse: bool = True, want_density: bool = True):
-    """Sol-Attn forward (solattn_forward). Returns (out, lse, density)."""
+RULES = {"threshold": _lib.RULE_THRESHOLD, "topk": _lib.RULE_TOPK, "topp": _lib.RULE_TOPP}
+
+
+def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, density=None, ws=None,
+            want_lse: bool = True, want_density: bool = True, rule: str = "threshold", topk: int = 0,
+            topp: float = 0.0, n_forced: int = 0):
+    """Sol-Attn forward. Returns (out, lse, density).
+
+    rule "threshold" (the method: tau_i = mu_i + beta sigma_i) calls
+    solattn_forward; "topk" / "topp" (ablation rules) or n_forced > 0 call
+    solattn_forward_ex."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
@@ -118,10 +126,19 @@ def forward(q, k, v, stats: PooledStats, beta: float, out=None, lse=None, densit
     if density is None and want_density:
         density = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
     ws = workspace(q.device) if ws is None else ws
-    rc = _lib.lib().solattn_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
-                                    ctypes.c_float(beta), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
-                                    ws.numel(), _stream())
-    _check(rc, "solattn_forward")
+    if rule == "threshold" and n_forced == 0:
+        rc = _lib.lib().solattn_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
+                                        ctypes.c_float(beta), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
+                                        ws.numel(), _stream())
+        _check(rc, "solattn_forward")
+    else:
+        if rule not in RULES:
+            raise ValueError(f"unknown rule {rule!r}")
+        opts = _lib.OptionsStruct(RULES[rule], float(beta), int(topk), float(topp), int(n_forced))
+        rc = _lib.lib().solattn_forward_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
+                                           ctypes.byref(opts), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
+                                           ws.numel(), _stream())
+        _check(rc, "solattn_forward_ex")
     return out, lse, density
 
 

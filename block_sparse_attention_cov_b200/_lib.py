@@ -16,6 +16,7 @@ EXPORTS = (
     "solattn_strerror",
     "solattn_version",
     "solattn_forward_noalloc",
+    "solattn_forward_ex",
 )
 
 OK = 0
@@ -31,12 +32,20 @@ WORKSPACE_BYTES = 256
 NOALLOC_SCRATCH_BYTES = 16 << 20
 BLOCK = 64
 MAX_TOKENS = 262144
+RULE_THRESHOLD, RULE_TOPK, RULE_TOPP = 0, 1, 2
 
 
 class PooledStruct(ctypes.Structure):
     """Mirror of solattn_pooled_t."""
 
     _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov")]
+
+
+class OptionsStruct(ctypes.Structure):
+    """Mirror of solattn_options_t."""
+
+    _fields_ = [("rule", ctypes.c_int), ("beta", ctypes.c_float), ("topk", ctypes.c_int), ("topp", ctypes.c_float),
+                ("n_forced", ctypes.c_int)]
 
 
 _lib = None
@@ -67,6 +76,9 @@ def lib() -> ctypes.CDLL:
     L.solattn_strerror.restype = ctypes.c_char_p
     L.solattn_forward_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
     L.solattn_forward_noalloc.restype = i
+    L.solattn_forward_ex.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(PooledStruct),
+                                     ctypes.POINTER(OptionsStruct), vp, vp, vp, vp, sz, vp]
+    L.solattn_forward_ex.restype = i
     L.solattn_version.argtypes = []
     L.solattn_version.restype = i
     _lib = L

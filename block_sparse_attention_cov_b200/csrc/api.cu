@@ -73,8 +73,9 @@ PooledPtrs to_ptrs(const solattn_pooled_t* p) {
 }
 
 int run_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
-                const solattn_pooled_t* pooled, float beta, bool route, void* out, float* lse, int32_t* density,
-                void* workspace, size_t workspace_bytes, void* stream) {
+                const solattn_pooled_t* pooled, const solattn_options_t& opt, bool route, void* out, float* lse,
+                int32_t* density, void* workspace, size_t workspace_bytes, void* stream) {
+  const float beta = opt.beta;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
   if ((rc = check_qkv(q, k, v))) return rc;
@@ -82,7 +83,9 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (!aligned16(out)) return SOLATTN_ERR_ALIGN;
   if ((lse && !aligned4(lse)) || (density && !aligned4(density))) return SOLATTN_ERR_ALIGN;
   if (route) {
-    if (std::isnan(beta)) return SOLATTN_ERR_ARG;
+    if (std::isnan(beta) || std::isnan(opt.topp) || opt.n_forced < 0) return SOLATTN_ERR_ARG;
+    if (opt.rule != SOLATTN_RULE_THRESHOLD && opt.rule != SOLATTN_RULE_TOPK && opt.rule != SOLATTN_RULE_TOPP)
+      return SOLATTN_ERR_ARG;
     if ((rc = check_pooled(pooled))) return rc;
   }
   if (!workspace || workspace_bytes < SOLATTN_WORKSPACE_BYTES) return SOLATTN_ERR_WORKSPACE;
@@ -101,6 +104,10 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   a.density = route ? density : nullptr;
   if (route) a.pooled = to_ptrs(pooled);
   a.beta = beta;
+  a.rule = route ? opt.rule : SOLATTN_RULE_THRESHOLD;
+  a.topk = opt.topk;
+  a.topp = opt.topp;
+  a.n_forced = route ? opt.n_forced : 0;
   a.route = route;
   a.BH = B * H;
   a.N = N;
@@ -179,14 +186,24 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
 int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                     const solattn_pooled_t* pooled, float beta, void* out, float* lse, int32_t* density_out,
                     void* workspace, size_t workspace_bytes, void* stream) {
-  return run_forward(q, k, v, B, H, N, d, pooled, beta, true, out, lse, density_out, workspace, workspace_bytes,
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0};
+  return run_forward(q, k, v, B, H, N, d, pooled, opt, true, out, lse, density_out, workspace, workspace_bytes,
+                     stream);
+}
+
+int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                       const solattn_pooled_t* pooled, const solattn_options_t* opts, void* out, float* lse,
+                       int32_t* density_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!opts) return SOLATTN_ERR_ARG;
+  return run_forward(q, k, v, B, H, N, d, pooled, *opts, true, out, lse, density_out, workspace, workspace_bytes,
                      stream);
 }
 
 int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int N, int d, void* out, float* lse,
                   void* workspace, size_t workspace_bytes, void* stream) {
-  return run_forward(q, k, v, B, H, N, d, nullptr, -INFINITY, false, out, lse, nullptr, workspace,
-                     workspace_bytes, stream);
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, -INFINITY, 0, 0.f, 0};
+  return run_forward(q, k, v, B, H, N, d, nullptr, opt, false, out, lse, nullptr, workspace, workspace_bytes,
+                     stream);
 }
 
 int solattn_status(const void* workspace, void* stream) {

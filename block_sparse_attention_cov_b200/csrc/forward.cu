@@ -85,12 +85,14 @@ enum : uint32_t {
   kSitePvDone,
 };
 
-template <int D>
+template <int D, bool SEL = false>
 struct __align__(1024) Smem {
   // K ring: one stage per 128-key tile (two blocks stacked in every 64-column
   // panel, as one N = 128 operand); V ring: one stage per block. Sizes are
   // multiples of 1 KB, so every stage stays 1024-aligned for the swizzle.
-  static constexpr int kKStages = D == 128 ? 3 : 4;
+  // (with a top-k / top-p rule the proxy rows of the unit are kept in shared
+  // memory for the selection, and the K ring gives up a stage for them)
+  static constexpr int kKStages = D == 128 ? (SEL ? 2 : 3) : 4;
   static constexpr int kVStages = D == 128 ? 4 : 8;
   uint8_t qt[kBM * D * 2];               // Q tile of the unit, SW128 K-major panels of 128 rows
   uint8_t kt[kKStages][kBM * D * 2];     // K tiles, same layout
@@ -110,6 +112,9 @@ struct __align__(1024) Smem {
   float rden[2];                     // running correction denominators
   int rkept[2];                      // running kept counts
   uint32_t bits[2][2][kNbMax / 32];  // kept bitmaps [slot][query block][word]: the unit's key list
+  float score[SEL ? 2 : 1][SEL ? kNbMax : 1];  // top-k / top-p: the unit's two proxy rows
+  uint32_t cut[2];                   // top-k / top-p: order key of each row's cut
+  int keep_none[2];                  // top-k / top-p: the row keeps no block by its rule
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   // Per S slot: QK landed / P stored by all four softmax warps / PV of the
   // slot's tile completed. Per-slot barriers keep a warp that runs a tile
@@ -131,6 +136,8 @@ struct __align__(1024) Smem {
 // one extra KB pays for the 1024-byte alignment of the TMA tiles.
 static_assert(sizeof(Smem<128>) + 1024 <= 232448, "shared memory layout too large");
 static_assert(sizeof(Smem<64>) + 1024 <= 232448, "shared memory layout too large");
+static_assert(sizeof(Smem<128, true>) + 1024 <= 232448, "shared memory layout too large");
+static_assert(sizeof(Smem<64, true>) + 1024 <= 232448, "shared memory layout too large");
 
 struct Params {
   const uint16_t* q;
@@ -143,6 +150,9 @@ struct Params {
   const float* kmean;
   const float* kcov;
   float beta;
+  int topk;         // top-k rule
+  float topp;       // top-p rule
+  int n_forced;     // leading key blocks always kept
   int BH, N, NB, npairs, units;
   DeviceStatus* status;
 };
@@ -171,8 +181,24 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
 }
 
 // Returns false if a bounded wait gave up (the CTA is aborting).
-template <int D>
-__device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair, int rt, uint32_t& chunk_ctr,
+// Order-preserving map of a float to an unsigned key (x < y <=> key(x) < key(y)).
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// RULE 0: per-row threshold tau_i = mu_i + beta sigma_i, decided chunk by
+// chunk as the scores are produced. RULE 1 / 2 (top-k / top-p): a first pass
+// stores the unit's two proxy rows, each row's cut is found by bisection on
+// the order keys, and a second pass decides and folds the corrections.
+template <int D, int RULE>
+__device__ bool route_unit(Smem<D, RULE != 0>& sm, const Params& P, int s, int bh, int pair, int rt, uint32_t& chunk_ctr,
                            volatile int* abort_flag, DeviceStatus* st, int u) {
   constexpr int VPL = D / 32;  // columns per lane in the scoring layout
   const int rw = rt / 32, lane = rt % 32;
@@ -210,7 +236,7 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   // row (every score equals mu_i = tau_i): nothing is strictly above it, so no
   // block is kept, whatever rounding does to the individual scores.
   float tau0 = beta, tau1 = has1 ? beta : INFINITY;
-  if (beta != -INFINITY && beta != INFINITY) {
+  if (RULE == 0 && beta != -INFINITY && beta != INFINITY) {
     // D = 128: thread rt owns column rt of both blocks; D = 64: column rt % 64
     // of block rt / 64. y_b[c] = sum_r C[r][c] qbar_b[r] (C is symmetric).
     const int col = rt % D, b1 = rt / D;
@@ -278,13 +304,22 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
   for (int a = 0; a < NACC; ++a) acc[a] = 0.f;
 
   bool ok = true;
+  constexpr bool SEL = RULE != 0;
+  for (int pass = SEL ? 0 : 1; pass < 2 && ok; ++pass) {
+  const bool scoring = !SEL || pass == 0;  // scores computed from the streamed pooled keys
+  const bool deciding = pass == 1;         // kept bits and corrections
   for (int c = 0; c < nchunks; ++c) {
     const uint32_t g = chunk_ctr + c, buf = g & 1;
-    if (rt == 0 && c + 1 < nchunks) issue(c + 1);  // buffer (c+1)&1 was released by chunk c-1
     float vcur[kChunk];
+    if (deciding) {
 #pragma unroll
-    for (int jj = 0; jj < kChunk; ++jj)
-      vcur[jj] = (c * kChunk + jj < NB) ? __ldg(vb + static_cast<long long>(c * kChunk + jj) * D + vcol) : 0.f;
+      for (int jj = 0; jj < kChunk; ++jj)
+        vcur[jj] = (c * kChunk + jj < NB) ? __ldg(vb + static_cast<long long>(c * kChunk + jj) * D + vcol) : 0.f;
+    }
+    const int j0 = c * kChunk;
+    const int nk = min(kChunk, NB - j0);
+    if (scoring) {
+    if (rt == 0 && c + 1 < nchunks) issue(c + 1);  // buffer (c+1)&1 was released by chunk c-1
     const bool landed = mbar_wait(&sm.rfull[buf], (g >> 1) & 1, abort_flag, st, kSiteRouteChunk, u);
     if (named_bar_or(1, 128, !landed || *abort_flag)) {
       // aborting: let the copies already issued (chunks c and c + 1) land first
@@ -295,8 +330,6 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
       ok = false;
       break;
     }
-    const int j0 = c * kChunk;
-    const int nk = min(kChunk, NB - j0);
     // ---- scores: warp rw handles key blocks 4 rw .. 4 rw + 3 of the chunk
     float v[8];
 #pragma unroll
@@ -345,14 +378,30 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     if ((lane & 3) == 0) {
       const int idx = lane >> 2;  // = 2 * kk + block
       sm.rscore[idx & 1][rw * 4 + (idx >> 1)] = v[0] * scale;
+      if constexpr (SEL) {
+        if (rw * 4 + (idx >> 1) < nk) sm.score[idx & 1][j0 + rw * 4 + (idx >> 1)] = v[0] * scale;
+      }
     }
     named_bar_sync(1, 128);
-    // ---- threshold, kept bits, correction weights (warp 0: block 0, warp 1: block 1)
+    }  // scoring
+    if (!deciding) {
+      named_bar_sync(1, 128);  // the chunk buffer is free again
+      continue;
+    }
+    // ---- kept bits, correction weights (warp 0: block 0, warp 1: block 1)
     if (rw < 2) {
       const int b = rw;
       const bool valid = lane < nk && (b == 0 || has1);
-      const float sh = sm.rscore[b][lane & (kChunk - 1)];
-      const bool kept = valid && sh > (b == 0 ? tau0 : tau1);
+      float sh;
+      bool by_rule;
+      if constexpr (SEL) {
+        sh = sm.score[b][j0 + (lane < nk ? lane : 0)];
+        by_rule = !sm.keep_none[b] && order_key(sh) >= sm.cut[b];
+      } else {
+        sh = sm.rscore[b][lane & (kChunk - 1)];
+        by_rule = sh > (b == 0 ? tau0 : tau1);
+      }
+      const bool kept = valid && (by_rule || j0 + lane < P.n_forced);
       const bool skip = valid && !kept;
       const uint32_t kmask = __ballot_sync(0xffffffffu, kept);
       float mx = skip ? sh : -INFINITY;
@@ -399,7 +448,65 @@ __device__ bool route_unit(Smem<D>& sm, const Params& P, int s, int bh, int pair
     }
     named_bar_sync(1, 128);  // chunk buffer and scratch free again
   }
-  chunk_ctr += nchunks;
+  if (scoring) chunk_ctr += nchunks;
+  if (SEL && pass == 0 && ok) {
+    // ---- each row's cut: the largest order key K whose superlevel set
+    // {j : key(s_hat_ij) >= K} still holds k blocks (top-k) or a fraction p of
+    // the row's mass sum_j n_j e^{s_hat_ij} (top-p); bisection over the 32 key
+    // bits, sums in a fixed order (warp 0: block 0, warp 1: block 1)
+    if (rw < 2) {
+      const int b = rw;
+      uint32_t K = 0u;
+      int none = (b == 1 && !has1) ? 1 : 0;
+      if (!none) {
+        if constexpr (RULE == 1) {
+          const int kk = P.topk;
+          if (kk <= 0) {
+            none = 1;
+          } else if (kk < NB) {
+            for (int bit = 31; bit >= 0; --bit) {
+              const uint32_t cand = K | (1u << bit);
+              int cnt = 0;
+              for (int j = lane; j < NB; j += 32) cnt += order_key(sm.score[b][j]) >= cand ? 1 : 0;
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+              if (cnt >= kk) K = cand;
+            }
+          }
+        } else {
+          const float p = P.topp;
+          if (p <= 0.f) {
+            none = 1;
+          } else if (p < 1.f) {
+            float M = -INFINITY;
+            for (int j = lane; j < NB; j += 32) M = fmaxf(M, sm.score[b][j]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            auto mass_at_least = [&](uint32_t cand) {
+              float w = 0.f;
+              for (int j = lane; j < NB; j += 32) {
+                const float sh = sm.score[b][j];
+                if (order_key(sh) >= cand)
+                  w += static_cast<float>(j == NB - 1 ? nlast : kBN) * ex2_approx((sh - M) * kLog2e);
+              }
+              return warp_sum(w);
+            };
+            const float target = p * mass_at_least(0u);
+            for (int bit = 31; bit >= 0; --bit) {
+              const uint32_t cand = K | (1u << bit);
+              if (mass_at_least(cand) >= target) K = cand;
+            }
+          }
+        }
+      }
+      if (lane == 0) {
+        sm.cut[b] = K;
+        sm.keep_none[b] = none;
+      }
+    }
+    named_bar_sync(1, 128);
+  }
+  }  // passes
   if (!ok) return false;
   // ---- publish the unit's correction and kept list into slot s
   if constexpr (D == 128) {
@@ -582,15 +689,16 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
 // tile is written over the first 64 columns of its own S) and O at 384. The
 // QKs of the next two tiles are in flight while the softmax works on one.
 // ---------------------------------------------------------------------------
-template <int D, bool ROUTE>
+template <int D, bool ROUTE, int RULE>
 __global__ void __launch_bounds__(kThreads, 1)
     solattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params P) {
-  constexpr int KS = Smem<D>::kKStages, VS = Smem<D>::kVStages;
+  using SmemT = Smem<D, RULE != 0>;
+  constexpr int KS = SmemT::kKStages, VS = SmemT::kVStages;
   constexpr uint32_t kColO = 3 * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* aligned = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  Smem<D>& sm = *reinterpret_cast<Smem<D>*>(aligned);
+  SmemT& sm = *reinterpret_cast<SmemT*>(aligned);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   DeviceStatus* st = P.status;
   volatile int* abort_flag = &sm.abort_flag;
@@ -664,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bh = u / P.npairs, pair = u % P.npairs;
       SOLATTN_TRACE_EVENT(13, rt == 0 ? n : 4096);
       if constexpr (ROUTE) {
-        if (!route_unit<D>(sm, P, s, bh, pair, rt, chunk_ctr, abort_flag, st, u)) break;
+        if (!route_unit<D, RULE>(sm, P, s, bh, pair, rt, chunk_ctr, abort_flag, st, u)) break;
       } else {
         if (rt == 0) {
           sm.count[s] = P.NB;
@@ -1066,7 +1174,7 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int rows
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool ROUTE>
+template <int D, bool ROUTE, int RULE>
 cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   CUtensorMap tmQ, tmK, tmV;
   if (!make_map(&tmQ, a.q, a.BH, a.N, D, kBM) || !make_map(&tmK, a.k, a.BH, a.N, D, kBN) ||
@@ -1083,18 +1191,21 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
   p.kmean = a.pooled.kmean;
   p.kcov = a.pooled.kcov;
   p.beta = a.beta;
+  p.topk = a.topk;
+  p.topp = a.topp;
+  p.n_forced = a.n_forced;
   p.BH = a.BH;
   p.N = a.N;
   p.NB = (a.N + kBN - 1) / kBN;
   p.npairs = (p.NB + 1) / 2;
   p.units = a.BH * p.npairs;
   p.status = static_cast<DeviceStatus*>(a.status);
-  const size_t smem = sizeof(Smem<D>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(solattn_fwd_kernel<D, ROUTE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = sizeof(Smem<D, RULE != 0>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(solattn_fwd_kernel<D, ROUTE, RULE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.units < num_sms ? p.units : num_sms;
-  solattn_fwd_kernel<D, ROUTE><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  solattn_fwd_kernel<D, ROUTE, RULE><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
@@ -1107,8 +1218,16 @@ extern "C" int solattn_trace_read(unsigned long long* host, size_t n) {
 #endif
 
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
-  if (a.d == 64) return a.route ? launch_fwd_t<64, true>(a, num_sms, stream) : launch_fwd_t<64, false>(a, num_sms, stream);
-  return a.route ? launch_fwd_t<128, true>(a, num_sms, stream) : launch_fwd_t<128, false>(a, num_sms, stream);
+  if (a.d == 64) {
+    if (!a.route) return launch_fwd_t<64, false, 0>(a, num_sms, stream);
+    if (a.rule == 1) return launch_fwd_t<64, true, 1>(a, num_sms, stream);
+    if (a.rule == 2) return launch_fwd_t<64, true, 2>(a, num_sms, stream);
+    return launch_fwd_t<64, true, 0>(a, num_sms, stream);
+  }
+  if (!a.route) return launch_fwd_t<128, false, 0>(a, num_sms, stream);
+  if (a.rule == 1) return launch_fwd_t<128, true, 1>(a, num_sms, stream);
+  if (a.rule == 2) return launch_fwd_t<128, true, 2>(a, num_sms, stream);
+  return launch_fwd_t<128, true, 0>(a, num_sms, stream);
 }
 
 }  // namespace solattn

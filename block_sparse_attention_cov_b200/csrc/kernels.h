@@ -24,6 +24,10 @@ struct ForwardArgs {
   int32_t* density;    // may be null
   PooledPtrs pooled;   // unused when route == false
   float beta;
+  int rule;            // 0 threshold, 1 top-k, 2 top-p (solattn_rule)
+  int topk;
+  float topp;
+  int n_forced;        // leading key blocks always kept
   bool route;          // false: dense attention (no routing, no correction)
   int BH, N, d;
   void* status;        // DeviceStatus in the caller's workspace

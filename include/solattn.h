@@ -130,6 +130,49 @@ int solattn_forward(const void* q, const void* k, const void* v, int B, int H, i
                     int32_t* density_out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Kept-set rules other than the per-row threshold, and always-kept blocks.
+ * The pages compare the threshold with the top-k and top-p routing of earlier
+ * methods (paithon.it, "Una soglia per ogni riga": a shared budget or a sort
+ * per row; "I numeri": routing time of threshold vs top-k vs top-p) and keep
+ * the text tokens of joint attention exact ("Dove leggere con attenzione"):
+ *   SOLATTN_RULE_THRESHOLD  S_i = {j : s_hat_ij > mu_i + beta sigma_i}
+ *   SOLATTN_RULE_TOPK       S_i = {j : s_hat_ij >= the topk-th largest s_hat_i.}
+ *                           (topk clamped to [0, N_b]; equal scores at the cut
+ *                           are all kept)
+ *   SOLATTN_RULE_TOPP       S_i = {j : s_hat_ij >= v*_i}, v*_i the largest score
+ *                           whose superlevel set carries a fraction >= topp of
+ *                           sum_j n_j e^{s_hat_ij}; topp <= 0 keeps nothing,
+ *                           topp >= 1 everything
+ * and in every rule blocks 0 .. n_forced - 1 are added to S_i. Skipped blocks
+ * get the same zeroth-order correction as with the threshold.
+ */
+enum solattn_rule {
+  SOLATTN_RULE_THRESHOLD = 0,
+  SOLATTN_RULE_TOPK = 1,
+  SOLATTN_RULE_TOPP = 2
+};
+
+typedef struct {
+  int rule;      /* enum solattn_rule */
+  float beta;    /* threshold rule (NaN rejected) */
+  int topk;      /* top-k rule: key blocks kept per query block */
+  float topp;    /* top-p rule: mass fraction (NaN rejected) */
+  int n_forced;  /* leading key blocks always kept, >= 0 (0 = none) */
+} solattn_options_t;
+
+/*
+ * solattn_forward with the kept-set rule and forced blocks of *opts (host
+ * memory, read during the call). solattn_forward(..., beta, ...) equals this
+ * call with {SOLATTN_RULE_THRESHOLD, beta, 0, 0, 0}. Errors as for
+ * solattn_forward, plus SOLATTN_ERR_ARG for a null opts, an unknown rule, a
+ * NaN beta/topp or a negative n_forced.
+ */
+int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                       const solattn_pooled_t* pooled, const solattn_options_t* opts, void* out,
+                       float* lse, int32_t* density_out, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
  * Dense softmax attention with scale 1/sqrt(d) by the same kernel with routing
  * switched off: equal to solattn_forward with beta = -INFINITY, without the
  * pooled statistics. lse may be NULL. workspace as for solattn_forward.

@@ -80,6 +80,23 @@ def test_forward_argument_errors(L):
     assert _fwd(L, wsb=255) == _lib.ERR_WORKSPACE
 
 
+def test_forward_ex_argument_errors(L):
+    def call(opts, **kw):
+        return L.solattn_forward_ex(FAKE, FAKE, FAKE, 1, 1, 128, 64, ctypes.byref(_pooled_struct()),
+                                    None if opts is None else ctypes.byref(opts), FAKE, None, None, FAKE, 256, None)
+    O = _lib.OptionsStruct
+    assert call(None) == _lib.ERR_ARG
+    assert call(O(7, 0.5, 0, 0.0, 0)) == _lib.ERR_ARG                      # unknown rule
+    assert call(O(_lib.RULE_THRESHOLD, math.nan, 0, 0.0, 0)) == _lib.ERR_ARG
+    assert call(O(_lib.RULE_TOPP, 0.0, 0, math.nan, 0)) == _lib.ERR_ARG
+    assert call(O(_lib.RULE_TOPK, 0.0, 3, 0.0, -1)) == _lib.ERR_ARG        # negative forced count
+    bad = _pooled_struct()
+    bad.kcov = None
+    assert L.solattn_forward_ex(FAKE, FAKE, FAKE, 1, 1, 128, 64, ctypes.byref(bad),
+                                ctypes.byref(O(_lib.RULE_TOPK, 0.0, 3, 0.0, 0)), FAKE, None, None, FAKE, 256,
+                                None) == _lib.ERR_ARG
+
+
 def test_dense_and_pool_argument_errors(L):
     assert L.solattn_dense(FAKE, FAKE, None, 1, 1, 64, 128, FAKE, None, FAKE, 256, None) == _lib.ERR_ARG
     assert L.solattn_dense(FAKE, FAKE, FAKE, 1, 1, 64, 32, FAKE, None, FAKE, 256, None) == _lib.ERR_UNSUPPORTED
