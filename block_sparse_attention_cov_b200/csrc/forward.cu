@@ -825,6 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           int jj[2];
           jj[0] = walk.next() & 0x3FFF;
           jj[1] = nb == 2 ? (walk.next() & 0x3FFF) : 0;
+#ifdef SOLATTN_TEST_HOOKS
+          if (gt == 0 && static_cast<int>(blockIdx.x) == g_hook_skip_cta) continue;  // this tile never arrives
+#endif
           if (elect_one()) {
             SOLATTN_TRACE_EVENT(15, gt);
             mbar_arrive_expect_tx(&sm.k_full[stg], nb * kBN * D * 2);
@@ -1210,6 +1213,16 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
 }
 
 }  // namespace
+
+#ifdef SOLATTN_TEST_HOOKS
+// Test builds only: CTA `skip_cta` never requests its first K tile (-1: none)
+// and every bounded wait gives up after `wait_budget_ns`.
+extern "C" int solattn_test_set_hook(int skip_cta, unsigned long long wait_budget_ns) {
+  if (cudaMemcpyToSymbol(g_hook_skip_cta, &skip_cta, sizeof(skip_cta)) != cudaSuccess) return 4;
+  if (cudaMemcpyToSymbol(g_wait_budget_ns, &wait_budget_ns, sizeof(wait_budget_ns)) != cudaSuccess) return 4;
+  return 0;
+}
+#endif
 
 #ifdef SOLATTN_TRACE
 extern "C" int solattn_trace_read(unsigned long long* host, size_t n) {

@@ -23,6 +23,17 @@ struct DeviceStatus {
 constexpr unsigned int kErrTimeout = 5;            // == SOLATTN_ERR_TIMEOUT
 constexpr unsigned long long kWaitBudgetNs = 2000000000ull;  // 2 s per wait
 
+#ifdef SOLATTN_TEST_HOOKS
+// Test builds only (a separate library used by the failure-detection tests):
+// the wait budget and a CTA whose first K tile is never requested can be set
+// from the host, so that a wait runs out on purpose, without any fault.
+static __device__ unsigned long long g_wait_budget_ns = kWaitBudgetNs;
+static __device__ int g_hook_skip_cta = -1;
+__device__ __forceinline__ unsigned long long wait_budget_ns() { return g_wait_budget_ns; }
+#else
+__device__ __forceinline__ unsigned long long wait_budget_ns() { return kWaitBudgetNs; }
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -106,7 +117,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitBudgetNs) {
+      if (global_timer_ns() - t0 > wait_budget_ns()) {
         if (atomicCAS(&st->error, 0u, kErrTimeout) == 0u) {
           st->where = site;
           st->unit = unit;
@@ -122,7 +133,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void mbar_wait_quiet(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitBudgetNs) return;
+    if (global_timer_ns() - t0 > wait_budget_ns()) return;
   }
 }
 
