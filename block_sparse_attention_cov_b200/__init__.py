@@ -42,11 +42,24 @@ def _shape(q: torch.Tensor):
 
 
 def _check_inputs(*ts):
+    """q, k, v (and out): CUDA bf16 [B, H, N, d] with contiguous d and one common
+    set of strides (contiguous, [B, N, H, d] seen through a permute, padded
+    rows, ...)."""
     for t in ts:
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
-            raise ValueError("q, k, v must be contiguous CUDA bf16 tensors [B, H, N, d]")
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.stride(-1) == 1):
+            raise ValueError("q, k, v must be CUDA bf16 [B, H, N, d] tensors with contiguous d")
     if not all(t.shape == ts[0].shape for t in ts):
         raise ValueError("q, k, v must have the same shape")
+    if not all(t.stride() == ts[0].stride() for t in ts):
+        raise ValueError("q, k, v must share their strides")
+
+
+def _strides(t):
+    """solattn_strides_t of a [B, H, N, d] tensor (all zero when contiguous)."""
+    if t.is_contiguous():
+        return _lib.StridesStruct(0, 0, 0)
+    sb, sh, sn, _ = t.stride()
+    return _lib.StridesStruct(sb, sh, sn)
 
 
 def _stream() -> ctypes.c_void_p:
@@ -96,8 +109,13 @@ def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stats: PooledStats |
         stats = PooledStats(buf, st, (B, H, N, d))
     elif stats.shape != (B, H, N, d):
         raise ValueError("PooledStats shape does not match the inputs")
-    _check(_lib.lib().solattn_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct), _stream()),
-           "solattn_pool")
+    if q.is_contiguous():
+        _check(_lib.lib().solattn_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
+                                       _stream()), "solattn_pool")
+    else:
+        strides = _strides(q)
+        _check(_lib.lib().solattn_pool_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(strides),
+                                          ctypes.byref(stats.struct), _stream()), "solattn_pool_ex")
     return stats
 
 
@@ -114,19 +132,22 @@ def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, 
             topp: float = 0.0, n_forced: int = 0):
     """Sol-Attn forward. Returns (out, lse, density).
 
-    rule "threshold" (the method: tau_i = mu_i + beta sigma_i) calls
-    solattn_forward; "topk" / "topp" (ablation rules) or n_forced > 0 call
-    solattn_forward_ex."""
+    rule "threshold" (the method: tau_i = mu_i + beta sigma_i) on contiguous
+    tensors calls solattn_forward; "topk" / "topp" (ablation rules),
+    n_forced > 0 or strided tensors call solattn_forward_ex. out is allocated
+    with q's strides (torch.empty_like) and must share them."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
     out = torch.empty_like(q) if out is None else out
+    if out.stride() != q.stride() or out.dtype != torch.bfloat16:
+        raise ValueError("out must be a bf16 tensor with q's strides")
     if lse is None and want_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if density is None and want_density:
         density = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
     ws = workspace(q.device) if ws is None else ws
-    if rule == "threshold" and n_forced == 0:
+    if rule == "threshold" and n_forced == 0 and q.is_contiguous():
         rc = _lib.lib().solattn_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
                                         ctypes.c_float(beta), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
                                         ws.numel(), _stream())
@@ -134,7 +155,7 @@ def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, 
     else:
         if rule not in RULES:
             raise ValueError(f"unknown rule {rule!r}")
-        opts = _lib.OptionsStruct(RULES[rule], float(beta), int(topk), float(topp), int(n_forced))
+        opts = _lib.OptionsStruct(RULES[rule], float(beta), int(topk), float(topp), int(n_forced), _strides(q))
         rc = _lib.lib().solattn_forward_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
                                            ctypes.byref(opts), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
                                            ws.numel(), _stream())

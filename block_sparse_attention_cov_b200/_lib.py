@@ -17,6 +17,7 @@ EXPORTS = (
     "solattn_version",
     "solattn_forward_noalloc",
     "solattn_forward_ex",
+    "solattn_pool_ex",
 )
 
 OK = 0
@@ -41,11 +42,17 @@ class PooledStruct(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov")]
 
 
+class StridesStruct(ctypes.Structure):
+    """Mirror of solattn_strides_t."""
+
+    _fields_ = [("batch", ctypes.c_longlong), ("head", ctypes.c_longlong), ("token", ctypes.c_longlong)]
+
+
 class OptionsStruct(ctypes.Structure):
     """Mirror of solattn_options_t."""
 
     _fields_ = [("rule", ctypes.c_int), ("beta", ctypes.c_float), ("topk", ctypes.c_int), ("topp", ctypes.c_float),
-                ("n_forced", ctypes.c_int)]
+                ("n_forced", ctypes.c_int), ("strides", StridesStruct)]
 
 
 _lib = None
@@ -79,6 +86,9 @@ def lib() -> ctypes.CDLL:
     L.solattn_forward_ex.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(PooledStruct),
                                      ctypes.POINTER(OptionsStruct), vp, vp, vp, vp, sz, vp]
     L.solattn_forward_ex.restype = i
+    L.solattn_pool_ex.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(StridesStruct), ctypes.POINTER(PooledStruct),
+                                  vp]
+    L.solattn_pool_ex.restype = i
     L.solattn_version.argtypes = []
     L.solattn_version.restype = i
     _lib = L

@@ -68,6 +68,20 @@ int current_device_sms(int* sms) {
   return SOLATTN_OK;
 }
 
+// Strides of q, k, v, out: all zero means contiguous [B][H][N][d]; otherwise
+// every stride a multiple of 8 elements (16 bytes: 128-bit loads, TMA) and the
+// token stride at least d.
+int resolve_strides(const solattn_strides_t* in, int H, int N, int d, solattn::Strides* out) {
+  if (!in || (in->batch == 0 && in->head == 0 && in->token == 0)) {
+    *out = solattn::Strides{static_cast<long long>(H) * N * d, static_cast<long long>(N) * d, d};
+    return SOLATTN_OK;
+  }
+  if (in->batch < 0 || in->head < 0 || in->token < d) return SOLATTN_ERR_ARG;
+  if ((in->batch | in->head | in->token) & 7) return SOLATTN_ERR_ARG;
+  *out = solattn::Strides{in->batch, in->head, in->token};
+  return SOLATTN_OK;
+}
+
 PooledPtrs to_ptrs(const solattn_pooled_t* p) {
   return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov};
 }
@@ -82,6 +96,8 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (!out) return SOLATTN_ERR_ARG;
   if (!aligned16(out)) return SOLATTN_ERR_ALIGN;
   if ((lse && !aligned4(lse)) || (density && !aligned4(density))) return SOLATTN_ERR_ALIGN;
+  solattn::Strides strides;
+  if ((rc = resolve_strides(&opt.strides, H, N, d, &strides))) return rc;
   if (route) {
     if (std::isnan(beta) || std::isnan(opt.topp) || opt.n_forced < 0) return SOLATTN_ERR_ARG;
     if (opt.rule != SOLATTN_RULE_THRESHOLD && opt.rule != SOLATTN_RULE_TOPK && opt.rule != SOLATTN_RULE_TOPP)
@@ -110,8 +126,10 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   a.n_forced = route ? opt.n_forced : 0;
   a.route = route;
   a.BH = B * H;
+  a.H = H;
   a.N = N;
   a.d = d;
+  a.st = strides;
   a.status = workspace;
   return solattn::launch_forward(a, sms, s) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
 }
@@ -170,15 +188,22 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
 
 int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                  const solattn_pooled_t* pooled, void* stream) {
+  return solattn_pool_ex(q, k, v, B, H, N, d, nullptr, pooled, stream);
+}
+
+int solattn_pool_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                    const solattn_strides_t* strides, const solattn_pooled_t* pooled, void* stream) {
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
+  solattn::Strides st;
+  if ((rc = resolve_strides(strides, H, N, d, &st))) return rc;
   if ((rc = check_qkv(q, k, v))) return rc;
   if ((rc = check_pooled(pooled))) return rc;
   int sms = 0;
   if ((rc = current_device_sms(&sms))) return rc;
   const cudaError_t e =
       solattn::launch_pool(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-                           static_cast<const uint16_t*>(v), to_ptrs(pooled), B * H, N, d, sms,
+                           static_cast<const uint16_t*>(v), to_ptrs(pooled), B * H, H, N, d, st, sms,
                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
 }
@@ -186,7 +211,7 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
 int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                     const solattn_pooled_t* pooled, float beta, void* out, float* lse, int32_t* density_out,
                     void* workspace, size_t workspace_bytes, void* stream) {
-  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0};
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0, {0, 0, 0}};
   return run_forward(q, k, v, B, H, N, d, pooled, opt, true, out, lse, density_out, workspace, workspace_bytes,
                      stream);
 }
@@ -201,7 +226,7 @@ int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H
 
 int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int N, int d, void* out, float* lse,
                   void* workspace, size_t workspace_bytes, void* stream) {
-  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, -INFINITY, 0, 0.f, 0};
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, -INFINITY, 0, 0.f, 0, {0, 0, 0}};
   return run_forward(q, k, v, B, H, N, d, nullptr, opt, false, out, lse, nullptr, workspace, workspace_bytes,
                      stream);
 }

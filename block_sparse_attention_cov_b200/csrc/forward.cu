@@ -153,7 +153,8 @@ struct Params {
   int topk;         // top-k rule
   float topp;       // top-p rule
   int n_forced;     // leading key blocks always kept
-  int BH, N, NB, npairs, units;
+  long long sb, sh, sn;  // element strides of q, k, v and out (batch, head, token)
+  int BH, H, N, NB, npairs, units;
   DeviceStatus* status;
 };
 
@@ -796,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sm.q_full, kBM * D * 2);
 #pragma unroll
           for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(&sm.qt[pnl * kBM * 128], &tmQ, &sm.q_full, pnl * 64, pair * kBM, bh);
+            tma_load_4d(&sm.qt[pnl * kBM * 128], &tmQ, &sm.q_full, pnl * 64, pair * kBM, bh % P.H, bh / P.H);
         }
       }
       if (named_bar_or(1, 128, !okq)) break;
@@ -834,8 +835,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int h = 0; h < nb; ++h) {
 #pragma unroll
               for (int pnl = 0; pnl < D / 64; ++pnl)
-                tma_load_3d(&sm.kt[stg][pnl * kBM * 128 + h * kBN * 128], &tmK, &sm.k_full[stg], pnl * 64,
-                            jj[h] * kBN, bh);
+                tma_load_4d(&sm.kt[stg][pnl * kBM * 128 + h * kBN * 128], &tmK, &sm.k_full[stg], pnl * 64,
+                            jj[h] * kBN, bh % P.H, bh / P.H);
             }
           }
           __syncwarp();
@@ -853,7 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.v_full[stg], kBN * D * 2);
 #pragma unroll
             for (int pnl = 0; pnl < D / 64; ++pnl)
-              tma_load_3d(&sm.vt[stg][pnl * kBN * 128], &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh);
+              tma_load_4d(&sm.vt[stg][pnl * kBN * 128], &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh % P.H,
+                          bh / P.H);
           }
           __syncwarp();
         }
@@ -1100,7 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = 1.f / L;
       const int row = pair * kBM + r;
       const bool valid = row < P.N;
-      uint16_t* orow = P.out + (static_cast<long long>(bh) * P.N + row) * D + hh * DH;
+      uint16_t* orow = P.out + (bh / P.H) * P.sb + (bh % P.H) * P.sh + static_cast<long long>(row) * P.sn + hh * DH;
 #pragma unroll 1
       for (int ch = 0; ch < DH / 16; ++ch) {
         float y[16];
@@ -1163,16 +1165,19 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH][N][D] bf16 viewed as a 3D tensor (D fastest); box = 64 columns x `rows`
-// rows, 128-byte swizzle; rows past N read as zero.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int rows) {
+// q, k or v as a 4D tensor {D, N, H, B} (D fastest) with the caller's element
+// strides; box = 64 columns x `rows` tokens of one (b, h), 128-byte swizzle;
+// tokens past N read as zero.
+bool make_map(CUtensorMap* map, const void* base, int B, int H, int N, int D, const Strides& st, int rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.n) * 2, static_cast<cuuint64_t>(st.h) * 2,
+                           static_cast<cuuint64_t>(st.b) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1180,8 +1185,9 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int rows
 template <int D, bool ROUTE, int RULE>
 cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   CUtensorMap tmQ, tmK, tmV;
-  if (!make_map(&tmQ, a.q, a.BH, a.N, D, kBM) || !make_map(&tmK, a.k, a.BH, a.N, D, kBN) ||
-      !make_map(&tmV, a.v, a.BH, a.N, D, kBN))
+  const int B = a.BH / a.H;
+  if (!make_map(&tmQ, a.q, B, a.H, a.N, D, a.st, kBM) || !make_map(&tmK, a.k, B, a.H, a.N, D, a.st, kBN) ||
+      !make_map(&tmV, a.v, B, a.H, a.N, D, a.st, kBN))
     return cudaErrorInvalidValue;
   Params p{};
   p.q = a.q;
@@ -1198,6 +1204,10 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
   p.topp = a.topp;
   p.n_forced = a.n_forced;
   p.BH = a.BH;
+  p.H = a.H;
+  p.sb = a.st.b;
+  p.sh = a.st.h;
+  p.sn = a.st.n;
   p.N = a.N;
   p.NB = (a.N + kBN - 1) / kBN;
   p.npairs = (p.NB + 1) / 2;

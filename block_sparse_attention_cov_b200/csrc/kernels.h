@@ -15,6 +15,11 @@ struct PooledPtrs {
   float* kcov;
 };
 
+// Element strides of q, k, v and out; the d elements of a token are contiguous.
+struct Strides {
+  long long b, h, n;
+};
+
 struct ForwardArgs {
   const uint16_t* q;
   const uint16_t* k;
@@ -29,12 +34,13 @@ struct ForwardArgs {
   float topp;
   int n_forced;        // leading key blocks always kept
   bool route;          // false: dense attention (no routing, no correction)
-  int BH, N, d;
+  int BH, H, N, d;
+  Strides st;          // of q, k, v and out
   void* status;        // DeviceStatus in the caller's workspace
 };
 
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, const PooledPtrs& p, int BH,
-                        int N, int d, int num_sms, cudaStream_t stream);
+                        int H, int N, int d, const Strides& st, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream);
 

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restr
                                                          const uint16_t* __restrict__ k,
                                                          const uint16_t* __restrict__ v, float* __restrict__ qbar,
                                                          float* __restrict__ kbar, float* __restrict__ vbar, int BH,
-                                                         int N, int NB) {
+                                                         int H, int N, int NB, Strides st) {
   constexpr int CH = D / 8;       // 16-byte chunks per row
   constexpr int RG = 256 / CH;    // row groups
   constexpr int RPT = kBlock / RG;  // rows per thread
@@ -69,12 +69,12 @@ __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restr
     float* dst = which == 0 ? qbar : (which == 1 ? kbar : vbar);
     const int row0 = j * kBlock;
     const int n = min(kBlock, N - row0);
-    const uint16_t* base = src + (static_cast<long long>(bh) * N + row0) * D + c * 8;
+    const uint16_t* base = src + (bh / H) * st.b + (bh % H) * st.h + static_cast<long long>(row0) * st.n + c * 8;
     uint4 w[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int row = g + r * RG;
-      w[r] = row < n ? ld_stream_v4(base + static_cast<long long>(row) * D) : make_uint4(0, 0, 0, 0);
+      w[r] = row < n ? ld_stream_v4(base + static_cast<long long>(row) * st.n) : make_uint4(0, 0, 0, 0);
     }
     float acc[8];
 #pragma unroll
@@ -261,11 +261,11 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(256)
 
 template <int D>
 cudaError_t launch_pool_d(const uint16_t* q, const uint16_t* k, const uint16_t* v, const PooledPtrs& p, int BH,
-                          int N, int num_sms, cudaStream_t stream) {
+                          int H, int N, const Strides& st, int num_sms, cudaStream_t stream) {
   const int NB = (N + kBlock - 1) / kBlock;
   const long long items = 3ll * BH * NB;
   const int grid1 = static_cast<int>(items < num_sms * 8ll ? items : num_sms * 8ll);
-  pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, BH, N, NB);
+  pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, BH, H, N, NB, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int smem = static_cast<int>(sizeof(KeyStatsSmem<D>));
@@ -278,9 +278,9 @@ cudaError_t launch_pool_d(const uint16_t* q, const uint16_t* k, const uint16_t* 
 }  // namespace
 
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, const PooledPtrs& p, int BH,
-                        int N, int d, int num_sms, cudaStream_t stream) {
-  if (d == 64) return launch_pool_d<64>(q, k, v, p, BH, N, num_sms, stream);
-  return launch_pool_d<128>(q, k, v, p, BH, N, num_sms, stream);
+                        int H, int N, int d, const Strides& st, int num_sms, cudaStream_t stream) {
+  if (d == 64) return launch_pool_d<64>(q, k, v, p, BH, H, N, st, num_sms, stream);
+  return launch_pool_d<128>(q, k, v, p, BH, H, N, st, num_sms, stream);
 }
 
 }  // namespace solattn

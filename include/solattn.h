@@ -100,6 +100,28 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
                  const solattn_pooled_t* pooled, void* stream);
 
 /*
+ * Element strides of q, k, v and out (the pages fix no layout): token (b, h, n)
+ * starts at b * batch + h * head + n * token elements from the base pointer and
+ * its d elements are contiguous. {H*N*d, N*d, d} is [B][H][N][d]; {N*H*d, d,
+ * H*d} is [B][N][H][d]. Every stride must be a multiple of 8 elements (16
+ * bytes) and token >= d; all zero means contiguous [B][H][N][d]. The four
+ * tensors share one set of strides.
+ */
+typedef struct {
+  long long batch;
+  long long head;
+  long long token;
+} solattn_strides_t;
+
+/*
+ * solattn_pool on q, k, v laid out with *strides (host memory, read during
+ * the call; NULL = contiguous). The pooled arrays are always contiguous.
+ * SOLATTN_ERR_ARG for strides that break the rules above.
+ */
+int solattn_pool_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                    const solattn_strides_t* strides, const solattn_pooled_t* pooled, void* stream);
+
+/*
  * Sol-Attn forward (hotpaper.ai abstract: routing, sparse computation and
  * correction in one online-softmax pass; paithon.it "Una soglia per ogni riga":
  * tau_i = mu_i + beta sigma_i, S_i = {j : s_hat_ij > tau_i}; "Scegliere mentre si
@@ -158,14 +180,15 @@ typedef struct {
   int topk;      /* top-k rule: key blocks kept per query block */
   float topp;    /* top-p rule: mass fraction (NaN rejected) */
   int n_forced;  /* leading key blocks always kept, >= 0 (0 = none) */
+  solattn_strides_t strides;  /* of q, k, v and out; all zero = contiguous [B][H][N][d] */
 } solattn_options_t;
 
 /*
- * solattn_forward with the kept-set rule and forced blocks of *opts (host
- * memory, read during the call). solattn_forward(..., beta, ...) equals this
- * call with {SOLATTN_RULE_THRESHOLD, beta, 0, 0, 0}. Errors as for
- * solattn_forward, plus SOLATTN_ERR_ARG for a null opts, an unknown rule, a
- * NaN beta/topp or a negative n_forced.
+ * solattn_forward with the kept-set rule, forced blocks and tensor strides of
+ * *opts (host memory, read during the call). solattn_forward(..., beta, ...)
+ * equals this call with {SOLATTN_RULE_THRESHOLD, beta, 0, 0, 0, {0, 0, 0}}.
+ * Errors as for solattn_forward, plus SOLATTN_ERR_ARG for a null opts, an
+ * unknown rule, a NaN beta/topp, a negative n_forced or invalid strides.
  */
 int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                        const solattn_pooled_t* pooled, const solattn_options_t* opts, void* out,

@@ -97,6 +97,22 @@ def test_forward_ex_argument_errors(L):
                                 None) == _lib.ERR_ARG
 
 
+def test_strides_validation(L):
+    S = _lib.StridesStruct
+    st = _pooled_struct()
+
+    def pool(strides):
+        return L.solattn_pool_ex(FAKE, FAKE, FAKE, 1, 2, 128, 64, ctypes.byref(strides), ctypes.byref(st), None)
+
+    def fwd(strides):
+        o = _lib.OptionsStruct(_lib.RULE_THRESHOLD, 0.5, 0, 0.0, 0, strides)
+        return L.solattn_forward_ex(FAKE, FAKE, FAKE, 1, 2, 128, 64, ctypes.byref(st), ctypes.byref(o), FAKE, None,
+                                    None, FAKE, 256, None)
+    for bad in (S(128 * 64 * 2, 64, 60), S(-8, 64, 128), S(128 * 128, 64 + 4, 128), S(0, 64 * 128, 32)):
+        assert pool(bad) == _lib.ERR_ARG
+        assert fwd(bad) == _lib.ERR_ARG
+
+
 def test_dense_and_pool_argument_errors(L):
     assert L.solattn_dense(FAKE, FAKE, None, 1, 1, 64, 128, FAKE, None, FAKE, 256, None) == _lib.ERR_ARG
     assert L.solattn_dense(FAKE, FAKE, FAKE, 1, 1, 64, 32, FAKE, None, FAKE, 256, None) == _lib.ERR_UNSUPPORTED
