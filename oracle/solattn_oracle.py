@@ -258,15 +258,21 @@ def route_rule(q: np.ndarray, k: np.ndarray, rule: str, param: float, n_forced: 
 # --------------------------------------------------------------------------
 # Step 6: attention with exact kept blocks and zeroth-order correction
 # --------------------------------------------------------------------------
-def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None):
+def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None, correction: str = "block"):
     """Sol-Attn forward for one head, offline threshold form.
 
     q, k, v: [N, d]. mask: optional [N_b, N_b] bool to use instead of the
     threshold (external-mask mode). rows: optional list of query-block indices
-    to compute (others are left NaN).
+    to compute (others are left NaN). correction: "block" (the library's
+    definition: a skipped block j reuses its proxy score s_hat_ij for every row
+    of block i) or "token" (the more literal reading of "Scegliere mentre si
+    calcola": every token of the skipped block is taken to carry the block's
+    mean key, so row t scores it s q_t . kbar_j; the value is still vbar_j).
     Returns out [N, d], lse [N] (natural log of the softmax denominator of the
     scaled scores), density [N_b] (= |S_i|).
     """
+    if correction not in ("block", "token"):
+        raise ValueError(correction)
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -277,6 +283,7 @@ def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None):
     r = route(q, k, beta)
     shat = r["shat"]
     vbar = pool(v)
+    kbar = r["kbar"]
     if mask is None:
         mask = r["mask"]
     mask = np.asarray(mask, dtype=bool)
@@ -290,7 +297,10 @@ def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None):
         skipped = np.nonzero(~mask[i])[0]
         tok = np.concatenate([np.arange(*bounds[j]) for j in kept]) if len(kept) else np.zeros(0, np.int64)
         scores = s * (qi @ k[tok].T)  # exact scores [n_i, tokens of kept blocks]
-        corr = np.broadcast_to(shat[i, skipped], (b - a, len(skipped)))  # proxy scores reused
+        if correction == "block":
+            corr = np.broadcast_to(shat[i, skipped], (b - a, len(skipped)))  # proxy scores reused
+        else:
+            corr = s * (qi @ kbar[skipped].T)  # each token against the skipped blocks' mean keys
         m = np.full((b - a,), -math.inf)
         if scores.shape[1]:
             m = np.maximum(m, scores.max(axis=1))
@@ -381,7 +391,7 @@ def _as64(t):
     return np.asarray(t, dtype=np.float64)
 
 
-def forward(q, k, v, beta: float = -math.inf, masks=None, rows=None):
+def forward(q, k, v, beta: float = -math.inf, masks=None, rows=None, correction: str = "block"):
     """attend() over every (b, h) of [B, H, N, d] inputs (torch or numpy).
 
     masks: optional [B, H, N_b, N_b] external masks. rows: optional query-block
@@ -397,7 +407,7 @@ def forward(q, k, v, beta: float = -math.inf, masks=None, rows=None):
     for b in range(B):
         for h in range(H):
             mk = None if masks is None else np.asarray(masks[b][h], bool)
-            out[b, h], lse[b, h], dens[b, h] = attend(q[b, h], k[b, h], v[b, h], beta, mk, rows)
+            out[b, h], lse[b, h], dens[b, h] = attend(q[b, h], k[b, h], v[b, h], beta, mk, rows, correction)
     return out, lse, dens
 
 

@@ -462,3 +462,65 @@ def test_planted_mistakes_in_the_other_rules_are_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_topk_keeps_exactly_the_k_largest(3)
     monkeypatch.undo()
+
+
+# ---------------------------------------------------------------------------
+# Per-token correction (the more literal reading of "Scegliere mentre si
+# calcola": each token of a skipped block carries the block's mean key)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("beta", [-0.5, 0.5, 1.5, math.inf])
+def test_token_correction_is_exact_for_key_block_constant_inputs(beta):
+    """Keys constant within each block: sum_u e^{s q_t.k_u} v_u over a skipped
+    block is n_j e^{s q_t.kbar_j} vbar_j exactly, so the per-token correction
+    reproduces dense attention (torch SDPA) for any beta, while the
+    block-level one does not (queries vary inside their blocks)."""
+    rng = _rng(51)
+    N, d = 64 * 5 + 23, 32
+    k = np.repeat(rng.standard_normal((6, d)), 64, axis=0)[:N]
+    q, v = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    ref = _sdpa64(q, k, v)
+    tok, _, _ = orc.attend(q, k, v, beta, correction="token")
+    np.testing.assert_allclose(tok, ref, rtol=1e-10, atol=1e-11)
+    blk, _, dens = orc.attend(q, k, v, beta, correction="block")
+    if (dens < 6).any():
+        assert np.abs(blk - ref).max() > 1e-3
+
+
+def test_token_correction_equals_block_for_query_block_constant_inputs():
+    rng = _rng(52)
+    N, d = 64 * 4 + 9, 32
+    q = np.repeat(rng.standard_normal((5, d)), 64, axis=0)[:N]
+    k, v = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    for beta in (0.0, 1.0, math.inf):
+        a, la, _ = orc.attend(q, k, v, beta, correction="token")
+        b, lb, _ = orc.attend(q, k, v, beta, correction="block")
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(la, lb, rtol=1e-12, atol=1e-13)
+
+
+def test_token_correction_brute_force_tiny():
+    rng = _rng(53)
+    N, d = 150, 16
+    q, k, v = (rng.standard_normal((N, d)) * 1.5 for _ in range(3))
+    beta = 0.4
+    out, lse, _ = orc.attend(q, k, v, beta, correction="token")
+    r = orc.route(q, k, beta)
+    bounds = orc.block_bounds(N)
+    s = 1 / math.sqrt(d)
+    for t in range(N):
+        i = t // 64
+        num, den, terms = np.zeros(d), 0.0, []
+        for j, (a, b) in enumerate(bounds):
+            if r["mask"][i, j]:
+                for u in range(a, b):
+                    terms.append((s * q[t] @ k[u], v[u]))
+            else:
+                kb, vb = k[a:b].mean(0), v[a:b].mean(0)
+                for _ in range(b - a):  # every token of the block, with the mean key and value
+                    terms.append((s * q[t] @ kb, vb))
+        m = max(x for x, _ in terms)
+        for x, vv in terms:
+            num += math.exp(x - m) * vv
+            den += math.exp(x - m)
+        np.testing.assert_allclose(out[t], num / den, rtol=1e-10, atol=1e-12)
+        assert abs(lse[t] - (m + math.log(den))) < 1e-10
