@@ -172,7 +172,7 @@ def dense_flops(B, H, N, d):
 
 def pool_bytes(B, H, N, d):
     nb = math.ceil(N / 64)
-    return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d) * B * H * 4
+    return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d) * B * H * 4 + 2 * nb * d * B * H * 2
 
 
 def cpu_threads():
@@ -277,7 +277,8 @@ def run_ours(args, rank, world, local_rank):
     nb = math.ceil(N / 64)
     dens = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
 
-    rule_kw = {"rule": args.rule, "topk": args.topk, "topp": args.topp, "n_forced": args.n_forced}
+    rule_kw = {"rule": args.rule, "topk": args.topk, "topp": args.topp, "n_forced": args.n_forced,
+               "correction": args.correction}
 
     def step(ev=None):
         if ev is not None:
@@ -414,6 +415,7 @@ def run_ours(args, rank, world, local_rank):
             "rule": args.rule, **({"topk": args.topk} if args.rule == "topk" else {}),
             **({"topp": args.topp} if args.rule == "topp" else {}),
             **({"n_forced": args.n_forced} if args.n_forced else {}),
+            **({"correction": args.correction} if args.correction != "block" else {}),
             "mean_density": mean_density, "global_batch": B * world, "seq_len": N,
             "parallelism": f"heads-independent replicas x{world}",
             "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no explicit flush" % (B * H * N * d * 2 / 1e6),
@@ -466,6 +468,8 @@ def main():
     ap.add_argument("--topp", type=float, default=0.1612,
                     help="top-p rule: mass fraction (0.1612 gives a 15 %% mean density on the Wan-like inputs)")
     ap.add_argument("--n-forced", type=int, default=0, help="leading key blocks always kept")
+    ap.add_argument("--correction", choices=["block", "token"], default="block",
+                    help="skipped-block correction: block-level proxy score (the method) or per token")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-dense", action="store_true")

@@ -89,11 +89,12 @@ class PooledStats:
         nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
         dims = {
             "qbar": (B, H, nb, d), "kbar": (B, H, nb, d), "vbar": (B, H, nb, d),
-            "kmean": (B, H, d), "kcov": (B, H, d, d),
+            "kmean": (B, H, d), "kcov": (B, H, d, d), "kbar16": (B, H, nb, d), "vbar16": (B, H, nb, d),
         }[name]
+        dt, size = (torch.bfloat16, 2) if name.endswith("16") else (torch.float32, 4)
         off = getattr(self.struct, name) - self.buffer.data_ptr()
         n = math.prod(dims)
-        return self.buffer[off:off + 4 * n].view(torch.float32).view(dims)
+        return self.buffer[off:off + size * n].view(dt).view(dims)
 
 
 def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stats: PooledStats | None = None) -> PooledStats:
@@ -129,13 +130,14 @@ RULES = {"threshold": _lib.RULE_THRESHOLD, "topk": _lib.RULE_TOPK, "topp": _lib.
 
 def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, density=None, ws=None,
             want_lse: bool = True, want_density: bool = True, rule: str = "threshold", topk: int = 0,
-            topp: float = 0.0, n_forced: int = 0):
+            topp: float = 0.0, n_forced: int = 0, correction: str = "block"):
     """Sol-Attn forward. Returns (out, lse, density).
 
     rule "threshold" (the method: tau_i = mu_i + beta sigma_i) on contiguous
     tensors calls solattn_forward; "topk" / "topp" (ablation rules),
-    n_forced > 0 or strided tensors call solattn_forward_ex. out is allocated
-    with q's strides (torch.empty_like) and must share them."""
+    n_forced > 0, strided tensors or correction="token" (skipped blocks scored
+    per query token against their mean key) call solattn_forward_ex. out is
+    allocated with q's strides (torch.empty_like) and must share them."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
@@ -147,7 +149,9 @@ def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, 
     if density is None and want_density:
         density = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
     ws = workspace(q.device) if ws is None else ws
-    if rule == "threshold" and n_forced == 0 and q.is_contiguous():
+    if correction not in ("block", "token"):
+        raise ValueError(f"unknown correction {correction!r}")
+    if rule == "threshold" and n_forced == 0 and q.is_contiguous() and correction == "block":
         rc = _lib.lib().solattn_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
                                         ctypes.c_float(beta), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
                                         ws.numel(), _stream())
@@ -155,7 +159,8 @@ def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, 
     else:
         if rule not in RULES:
             raise ValueError(f"unknown rule {rule!r}")
-        opts = _lib.OptionsStruct(RULES[rule], float(beta), int(topk), float(topp), int(n_forced), _strides(q))
+        opts = _lib.OptionsStruct(RULES[rule], float(beta), int(topk), float(topp), int(n_forced), _strides(q),
+                                  1 if correction == "token" else 0)
         rc = _lib.lib().solattn_forward_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.byref(stats.struct),
                                            ctypes.byref(opts), _ptr(out), _ptr(lse), _ptr(density), _ptr(ws),
                                            ws.numel(), _stream())

@@ -39,7 +39,7 @@ RULE_THRESHOLD, RULE_TOPK, RULE_TOPP = 0, 1, 2
 class PooledStruct(ctypes.Structure):
     """Mirror of solattn_pooled_t."""
 
-    _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov")]
+    _fields_ = [(name, ctypes.c_void_p) for name in ("qbar", "kbar", "vbar", "kmean", "kcov", "kbar16", "vbar16")]
 
 
 class StridesStruct(ctypes.Structure):
@@ -52,7 +52,7 @@ class OptionsStruct(ctypes.Structure):
     """Mirror of solattn_options_t."""
 
     _fields_ = [("rule", ctypes.c_int), ("beta", ctypes.c_float), ("topk", ctypes.c_int), ("topp", ctypes.c_float),
-                ("n_forced", ctypes.c_int), ("strides", StridesStruct)]
+                ("n_forced", ctypes.c_int), ("strides", StridesStruct), ("correction", ctypes.c_int)]
 
 
 _lib = None

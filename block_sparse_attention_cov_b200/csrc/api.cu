@@ -41,7 +41,7 @@ int check_qkv(const void* q, const void* k, const void* v) {
 
 int check_pooled(const solattn_pooled_t* p) {
   if (!p) return SOLATTN_ERR_ARG;
-  const void* ptrs[5] = {p->qbar, p->kbar, p->vbar, p->kmean, p->kcov};
+  const void* ptrs[7] = {p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, p->kbar16, p->vbar16};
   for (const void* x : ptrs)
     if (!x) return SOLATTN_ERR_ARG;
   for (const void* x : ptrs)
@@ -83,7 +83,8 @@ int resolve_strides(const solattn_strides_t* in, int H, int N, int d, solattn::S
 }
 
 PooledPtrs to_ptrs(const solattn_pooled_t* p) {
-  return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov};
+  return PooledPtrs{p->qbar, p->kbar, p->vbar, p->kmean, p->kcov, static_cast<uint16_t*>(p->kbar16),
+                    static_cast<uint16_t*>(p->vbar16)};
 }
 
 int run_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
@@ -102,6 +103,7 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
     if (std::isnan(beta) || std::isnan(opt.topp) || opt.n_forced < 0) return SOLATTN_ERR_ARG;
     if (opt.rule != SOLATTN_RULE_THRESHOLD && opt.rule != SOLATTN_RULE_TOPK && opt.rule != SOLATTN_RULE_TOPP)
       return SOLATTN_ERR_ARG;
+    if (opt.correction != 0 && opt.correction != 1) return SOLATTN_ERR_ARG;
     if ((rc = check_pooled(pooled))) return rc;
   }
   if (!workspace || workspace_bytes < SOLATTN_WORKSPACE_BYTES) return SOLATTN_ERR_WORKSPACE;
@@ -124,6 +126,7 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   a.topk = opt.topk;
   a.topp = opt.topp;
   a.n_forced = route ? opt.n_forced : 0;
+  a.token_corr = route ? opt.correction : 0;
   a.route = route;
   a.BH = B * H;
   a.H = H;
@@ -164,10 +167,10 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t nb = (static_cast<size_t>(N) + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
   const size_t f = sizeof(float);
-  const size_t sizes[5] = {bh * nb * d * f, bh * nb * d * f, bh * nb * d * f, bh * d * f,
-                           bh * static_cast<size_t>(d) * d * f};
-  size_t off[5], total = 0;
-  for (int i = 0; i < 5; ++i) {
+  const size_t sizes[7] = {bh * nb * d * f, bh * nb * d * f, bh * nb * d * f, bh * d * f,
+                           bh * static_cast<size_t>(d) * d * f, bh * nb * d * 2, bh * nb * d * 2};
+  size_t off[7], total = 0;
+  for (int i = 0; i < 7; ++i) {
     off[i] = total;
     total += round256(sizes[i]);
   }
@@ -180,6 +183,8 @@ int solattn_pooled_layout(int B, int H, int N, int d, void* base, solattn_pooled
     pooled->vbar = reinterpret_cast<float*>(b + off[2]);
     pooled->kmean = reinterpret_cast<float*>(b + off[3]);
     pooled->kcov = reinterpret_cast<float*>(b + off[4]);
+    pooled->kbar16 = b + off[5];
+    pooled->vbar16 = b + off[6];
   } else if (pooled && !base) {
     return SOLATTN_ERR_ARG;
   }
@@ -211,7 +216,7 @@ int solattn_pool_ex(const void* q, const void* k, const void* v, int B, int H, i
 int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                     const solattn_pooled_t* pooled, float beta, void* out, float* lse, int32_t* density_out,
                     void* workspace, size_t workspace_bytes, void* stream) {
-  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0, {0, 0, 0}};
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0, {0, 0, 0}, 0};
   return run_forward(q, k, v, B, H, N, d, pooled, opt, true, out, lse, density_out, workspace, workspace_bytes,
                      stream);
 }
@@ -226,7 +231,7 @@ int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H
 
 int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int N, int d, void* out, float* lse,
                   void* workspace, size_t workspace_bytes, void* stream) {
-  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, -INFINITY, 0, 0.f, 0, {0, 0, 0}};
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, -INFINITY, 0, 0.f, 0, {0, 0, 0}, 0};
   return run_forward(q, k, v, B, H, N, d, nullptr, opt, false, out, lse, nullptr, workspace, workspace_bytes,
                      stream);
 }

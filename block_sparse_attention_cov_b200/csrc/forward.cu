@@ -153,6 +153,7 @@ struct Params {
   int topk;         // top-k rule
   float topp;       // top-p rule
   int n_forced;     // leading key blocks always kept
+  int token_corr;   // 1: skipped blocks attended per token as tiles of pooled keys
   long long sb, sh, sn;  // element strides of q, k, v and out (batch, head, token)
   int BH, H, N, NB, npairs, units;
   DeviceStatus* status;
@@ -672,6 +673,23 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
   }
 }
 
+// Tiles of a unit: TT of kept blocks (two per tile) and, with the per-token
+// correction, TP of pooled keys (128 per tile, every key block of the head;
+// columns are masked per query block to the blocks it skipped). V blocks: T
+// kept ones, then the 64-key chunks of the pooled values.
+struct UnitTiles {
+  int T, TT, TP, VB;
+  __device__ __forceinline__ UnitTiles(int T_, int NB, bool token)
+      : T(T_), TT((T_ + 1) / 2), TP(token ? (NB + 127) / 128 : 0), VB(T_ + (token ? (NB + 63) / 64 : 0)) {}
+  __device__ __forceinline__ int total() const { return TT + TP; }
+  // key blocks (64-key halves) in tile t
+  __device__ __forceinline__ int halves(int t, int NB) const {
+    return t < TT ? ((2 * t + 1 < T) ? 2 : 1) : ((128 * (t - TT) + 64 < NB) ? 2 : 1);
+  }
+  // index of half h of tile t among the unit's V blocks
+  __device__ __forceinline__ int vblock(int t, int h) const { return t < TT ? 2 * t + h : T + 2 * (t - TT) + h; }
+};
+
 // ---------------------------------------------------------------------------
 // The kernel. 512 threads = 16 warps:
 //   warps 0-7   softmax: warp w covers rows 32 (w % 4) .. + 31 of the unit
@@ -690,10 +708,11 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
 // tile is written over the first 64 columns of its own S) and O at 384. The
 // QKs of the next two tiles are in flight while the softmax works on one.
 // ---------------------------------------------------------------------------
-template <int D, bool ROUTE, int RULE>
+template <int D, bool ROUTE, int RULE, bool TOKEN>
 __global__ void __launch_bounds__(kThreads, 1)
     solattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const Params P) {
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+                       const __grid_constant__ CUtensorMap tmVb, const Params P) {
   using SmemT = Smem<D, RULE != 0>;
   constexpr int KS = SmemT::kKStages, VS = SmemT::kVStages;
   constexpr uint32_t kColO = 3 * 128;
@@ -740,6 +759,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
+    if (TOKEN) {
+      prefetch_tensormap(&tmKb);
+      prefetch_tensormap(&tmVb);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -816,16 +839,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bh = u / P.npairs;
       bool ok = true;
       KeyWalk<ROUTE> walk(sm.bits[s][0], sm.bits[s][1]);
+      const UnitTiles ut(T, P.NB, TOKEN);
       if (isK) {
-        const int TT = (T + 1) / 2;
+        const int TT = ut.total();
         int t = 0;
         for (; t < TT; ++t) {
           const uint32_t gt = g + t, stg = gt % KS, r = gt / KS;
           if (r >= 1 && !warp_wait(&sm.k_empty[stg], (r - 1) & 1, abort_flag, st, kSiteKEmpty, u)) break;
-          const int nb = (2 * t + 1 < T) ? 2 : 1;
+          const int nb = ut.halves(t, P.NB);
+          const bool pooled = TOKEN && t >= ut.TT;  // a tile of pooled keys (per-token correction)
           int jj[2];
-          jj[0] = walk.next() & 0x3FFF;
-          jj[1] = nb == 2 ? (walk.next() & 0x3FFF) : 0;
+          if (!pooled) {
+            jj[0] = walk.next() & 0x3FFF;
+            jj[1] = nb == 2 ? (walk.next() & 0x3FFF) : 0;
+          } else {
+            jj[0] = 2 * (t - ut.TT);
+            jj[1] = jj[0] + 1;
+          }
 #ifdef SOLATTN_TEST_HOOKS
           if (gt == 0 && static_cast<int>(blockIdx.x) == g_hook_skip_cta) continue;  // this tile never arrives
 #endif
@@ -834,9 +864,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.k_full[stg], nb * kBN * D * 2);
             for (int h = 0; h < nb; ++h) {
 #pragma unroll
-              for (int pnl = 0; pnl < D / 64; ++pnl)
-                tma_load_4d(&sm.kt[stg][pnl * kBM * 128 + h * kBN * 128], &tmK, &sm.k_full[stg], pnl * 64,
-                            jj[h] * kBN, bh % P.H, bh / P.H);
+              for (int pnl = 0; pnl < D / 64; ++pnl) {
+                void* dst = &sm.kt[stg][pnl * kBM * 128 + h * kBN * 128];
+                if (!pooled)
+                  tma_load_4d(dst, &tmK, &sm.k_full[stg], pnl * 64, jj[h] * kBN, bh % P.H, bh / P.H);
+                else  // rows 64 jj[h] .. of the head's bf16 pooled keys
+                  tma_load_4d(dst, &tmKb, &sm.k_full[stg], pnl * 64, jj[h] * kBN, 0, bh);
+              }
             }
           }
           __syncwarp();
@@ -845,22 +879,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = t == TT;
       } else {
         int t = 0;
-        for (; t < T; ++t) {
-          const int j = walk.next() & 0x3FFF;
+        for (; t < ut.VB; ++t) {
+          const bool pooled = TOKEN && t >= T;
+          const int j = pooled ? t - T : (walk.next() & 0x3FFF);
           const uint32_t gt = g + t, stg = gt % VS, r = gt / VS;
           if (r >= 1 && !warp_wait(&sm.v_empty[stg], (r - 1) & 1, abort_flag, st, kSiteVEmpty, u)) break;
           if (elect_one()) {
             SOLATTN_TRACE_EVENT(16, gt);
             mbar_arrive_expect_tx(&sm.v_full[stg], kBN * D * 2);
 #pragma unroll
-            for (int pnl = 0; pnl < D / 64; ++pnl)
-              tma_load_4d(&sm.vt[stg][pnl * kBN * 128], &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh % P.H,
-                          bh / P.H);
+            for (int pnl = 0; pnl < D / 64; ++pnl) {
+              void* dst = &sm.vt[stg][pnl * kBN * 128];
+              if (!pooled)
+                tma_load_4d(dst, &tmV, &sm.v_full[stg], pnl * 64, j * kBN, bh % P.H, bh / P.H);
+              else
+                tma_load_4d(dst, &tmVb, &sm.v_full[stg], pnl * 64, j * kBN, 0, bh);
+            }
           }
           __syncwarp();
         }
         g += t;
-        ok = t == T;
+        ok = t == ut.VB;
       }
       if (!ok) break;  // aborted
       if (elect_one()) mbar_arrive(&sm.route_empty[s]);
@@ -901,7 +940,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      const int TT = (T + 1) / 2;
+      const UnitTiles ut(T, P.NB, TOKEN);
+      const int TT = ut.total();
       if (isQK) {
         if (!warp_wait(&sm.q_full, n & 1, abort_flag, st, kSiteQFull, u)) break;
         if (TT == 0) {  // nothing to multiply: release the Q tile
@@ -918,7 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (elect_one()) {
             const uint64_t kd = kdesc0 + ((stg * (kBM * D * 2)) >> 4);
-            const uint32_t idesc = (2 * t + 1 < T) ? idesc_qk2 : idesc_qk1;
+            const uint32_t idesc = ut.halves(t, P.NB) == 2 ? idesc_qk2 : idesc_qk1;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (((kk / 4) * kBM * 128) + (kk % 4) * 32) >> 4;
@@ -936,12 +976,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n >= 1 && !warp_wait(&sm.o_free[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, st, kSiteOFree, u)) break;
         for (int t = 0; t < TT && ok; ++t) {
           const uint32_t gt = gtile + t;
-          const int nb = (2 * t + 1 < T) ? 2 : 1;
+          const int nb = ut.halves(t, P.NB);
           if (!warp_wait(&sm.p_full[gt % 3], (gt / 3) & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
           if (lane == 0) SOLATTN_TRACE_EVENT(12, gt);
           uint32_t stv[2];
           for (int h = 0; h < nb && ok; ++h) {
-            const uint32_t gv = gblk + 2 * t + h;
+            const uint32_t gv = gblk + ut.vblock(t, h);
             stv[h] = gv % VS;
             ok = warp_wait(&sm.v_full[stv[h]], (gv / VS) & 1, abort_flag, st, kSiteVFull, u);
           }
@@ -968,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) mma_commit(&sm.route_empty[s]);
       __syncwarp();
       gtile += TT;
-      gblk += T;
+      gblk += ut.VB;
     }
     const int me = isQK ? 0 : 1;
     if (elect_one()) mma_commit(&sm.mma_done[me]);  // teardown: issued MMAs complete before TMEM is freed
@@ -986,6 +1026,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nlast = P.N - (P.NB - 1) * kBN;
     constexpr int DH = D / 2;                 // O / output columns owned by this warp
     const uint32_t colO = tmem + kColO + lane_off + hh * DH;
+    // per-token correction: a pooled key stands for n_j tokens, log2(n_j) added
+    // to its score (in raw score units)
+    const float wfull = 6.f / sl2, wlast = __log2f(static_cast<float>(nlast)) / sl2;
     uint32_t gtile = 0;
     for (int n = 0;; ++n) {
       const int s = n & 1;
@@ -995,27 +1038,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = sm.unit[s];
       if (u < 0) break;
       const int T = sm.count[s];
-      const int TT = (T + 1) / 2;
+      const UnitTiles ut(T, P.NB, TOKEN);
+      const int TT = ut.total();
       float m = -INFINITY, l = 0.f;  // m: the row's shared reference max; l: this half's sum
       bool ok = true;
       KeyWalk<ROUTE> walk(sm.bits[s][0], sm.bits[s][1]);
       for (int t = 0; t < TT; ++t) {
         const uint32_t gt = gtile + t, slot = gt % 3;
         const uint32_t colS = tmem + slot * 128 + lane_off;
-        const int nb = (2 * t + 1 < T) ? 2 : 1;
-        uint32_t entry = 0u;
+        const int nb = ut.halves(t, P.NB);
+        const bool pooled = TOKEN && t >= ut.TT;
+        bool kept;
+        int nv = kBN;
+        uint64_t use = 0ull;  // pooled tile: this half's columns whose block this row's query block skipped
+        int j0 = 0;
+        if (!pooled) {
+          uint32_t entry = 0u;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t e = h < nb ? walk.next() : 0u;
-          if (h == hh) entry = e;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t e = h < nb ? walk.next() : 0u;
+            if (h == hh) entry = e;
+          }
+          kept = (entry >> (14 + blk)) & 1u;
+          nv = ((entry & 0x3FFF) == static_cast<uint32_t>(P.NB - 1)) ? nlast : kBN;
+        } else {
+          j0 = 128 * (t - ut.TT) + 64 * hh;  // first pooled key of this half (a multiple of 64)
+          if (hh < nb) {
+            const uint64_t kb = static_cast<uint64_t>(sm.bits[s][blk][j0 >> 5]) |
+                                (static_cast<uint64_t>(sm.bits[s][blk][(j0 >> 5) + 1]) << 32);
+            const int valid = min(64, P.NB - j0);
+            use = ~kb & (valid >= 64 ? ~0ull : ((1ull << valid) - 1ull));
+          }
+          kept = use != 0ull;
         }
-        const bool kept = (entry >> (14 + blk)) & 1u;
-        const int nv = ((entry & 0x3FFF) == static_cast<uint32_t>(P.NB - 1)) ? nlast : kBN;
         const bool okw = warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
         tc_fence_after();
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(0, gt);
         uint32_t sv[64];
         if (kept && okw) tmem_ld32x2_wait(colS + 64 * hh, colS + 64 * hh + 32, sv);
+        if (TOKEN && pooled && kept && okw) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float w = (j0 + c == P.NB - 1) ? wlast : wfull;
+            sv[c] = ((use >> c) & 1ull) ? __float_as_uint(__uint_as_float(sv[c]) + w) : 0xFF800000u;
+          }
+        }
         const float mx = (kept && okw) ? tile_max(sv, nv) * sl2 : -INFINITY;
         // Does a row of this group need a new reference max (or did a wait fail)?
         // The barrier also orders this group's S reads before the other half's
@@ -1093,7 +1160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float lrow = sm.xl[r][0] + sm.xl[r][1];
       named_bar_sync(pb, 64);  // both halves have read xl
-      const float mc = sm.cmax[s][blk] * kLog2e;
+      // (with the per-token correction the skipped blocks came in as pooled tiles)
+      const float mc = TOKEN ? -INFINITY : sm.cmax[s][blk] * kLog2e;
       const float cd = sm.cden[s][blk];
       const float mf = fmaxf(m, mc);
       const float wa = (m == -INFINITY) ? 0.f : ex2_approx(m - mf);
@@ -1182,13 +1250,22 @@ bool make_map(CUtensorMap* map, const void* base, int B, int H, int N, int D, co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool ROUTE, int RULE>
+template <int D, bool ROUTE, int RULE, bool TOKEN>
 cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   CUtensorMap tmQ, tmK, tmV;
   const int B = a.BH / a.H;
   if (!make_map(&tmQ, a.q, B, a.H, a.N, D, a.st, kBM) || !make_map(&tmK, a.k, B, a.H, a.N, D, a.st, kBN) ||
       !make_map(&tmV, a.v, B, a.H, a.N, D, a.st, kBN))
     return cudaErrorInvalidValue;
+  // bf16 pooled keys / values of every head, [BH][N_b][D], for the per-token correction
+  CUtensorMap tmKb = tmK, tmVb = tmV;
+  if (TOKEN) {
+    const int NB = (a.N + kBN - 1) / kBN;
+    const Strides ps{static_cast<long long>(NB) * D, static_cast<long long>(NB) * D, D};
+    if (!make_map(&tmKb, a.pooled.kbar16, a.BH, 1, NB, D, ps, kBN) ||
+        !make_map(&tmVb, a.pooled.vbar16, a.BH, 1, NB, D, ps, kBN))
+      return cudaErrorInvalidValue;
+  }
   Params p{};
   p.q = a.q;
   p.out = a.out;
@@ -1203,6 +1280,7 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
   p.topk = a.topk;
   p.topp = a.topp;
   p.n_forced = a.n_forced;
+  p.token_corr = a.token_corr;
   p.BH = a.BH;
   p.H = a.H;
   p.sb = a.st.b;
@@ -1214,11 +1292,11 @@ cudaError_t launch_fwd_t(const ForwardArgs& a, int num_sms, cudaStream_t stream)
   p.units = a.BH * p.npairs;
   p.status = static_cast<DeviceStatus*>(a.status);
   const size_t smem = sizeof(Smem<D, RULE != 0>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(solattn_fwd_kernel<D, ROUTE, RULE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(solattn_fwd_kernel<D, ROUTE, RULE, TOKEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.units < num_sms ? p.units : num_sms;
-  solattn_fwd_kernel<D, ROUTE, RULE><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  solattn_fwd_kernel<D, ROUTE, RULE, TOKEN><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, tmKb, tmVb, p);
   return cudaGetLastError();
 }
 
@@ -1240,17 +1318,25 @@ extern "C" int solattn_trace_read(unsigned long long* host, size_t n) {
 }
 #endif
 
+template <int D, bool ROUTE, int RULE>
+cudaError_t launch_fwd_c(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
+  if constexpr (ROUTE) {
+    if (a.token_corr) return launch_fwd_t<D, ROUTE, RULE, true>(a, num_sms, stream);
+  }
+  return launch_fwd_t<D, ROUTE, RULE, false>(a, num_sms, stream);
+}
+
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   if (a.d == 64) {
-    if (!a.route) return launch_fwd_t<64, false, 0>(a, num_sms, stream);
-    if (a.rule == 1) return launch_fwd_t<64, true, 1>(a, num_sms, stream);
-    if (a.rule == 2) return launch_fwd_t<64, true, 2>(a, num_sms, stream);
-    return launch_fwd_t<64, true, 0>(a, num_sms, stream);
+    if (!a.route) return launch_fwd_c<64, false, 0>(a, num_sms, stream);
+    if (a.rule == 1) return launch_fwd_c<64, true, 1>(a, num_sms, stream);
+    if (a.rule == 2) return launch_fwd_c<64, true, 2>(a, num_sms, stream);
+    return launch_fwd_c<64, true, 0>(a, num_sms, stream);
   }
-  if (!a.route) return launch_fwd_t<128, false, 0>(a, num_sms, stream);
-  if (a.rule == 1) return launch_fwd_t<128, true, 1>(a, num_sms, stream);
-  if (a.rule == 2) return launch_fwd_t<128, true, 2>(a, num_sms, stream);
-  return launch_fwd_t<128, true, 0>(a, num_sms, stream);
+  if (!a.route) return launch_fwd_c<128, false, 0>(a, num_sms, stream);
+  if (a.rule == 1) return launch_fwd_c<128, true, 1>(a, num_sms, stream);
+  if (a.rule == 2) return launch_fwd_c<128, true, 2>(a, num_sms, stream);
+  return launch_fwd_c<128, true, 0>(a, num_sms, stream);
 }
 
 }  // namespace solattn

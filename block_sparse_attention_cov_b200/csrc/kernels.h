@@ -13,6 +13,8 @@ struct PooledPtrs {
   float* vbar;
   float* kmean;
   float* kcov;
+  uint16_t* kbar16;  // bf16 copies for the per-token correction
+  uint16_t* vbar16;
 };
 
 // Element strides of q, k, v and out; the d elements of a token are contiguous.
@@ -33,6 +35,7 @@ struct ForwardArgs {
   int topk;
   float topp;
   int n_forced;        // leading key blocks always kept
+  int token_corr;      // 1: per-token correction through pooled-key tiles
   bool route;          // false: dense attention (no routing, no correction)
   int BH, H, N, d;
   Strides st;          // of q, k, v and out

@@ -15,6 +15,7 @@
 // The per-row statistics mu_i, sigma_i are evaluated by the forward kernel's
 // routing warps from kmean and kcov.
 #include <cooperative_groups.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -50,8 +51,9 @@ template <int D>
 __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restrict__ q,
                                                          const uint16_t* __restrict__ k,
                                                          const uint16_t* __restrict__ v, float* __restrict__ qbar,
-                                                         float* __restrict__ kbar, float* __restrict__ vbar, int BH,
-                                                         int H, int N, int NB, Strides st) {
+                                                         float* __restrict__ kbar, float* __restrict__ vbar,
+                                                         uint16_t* __restrict__ kbar16, uint16_t* __restrict__ vbar16,
+                                                         int BH, int H, int N, int NB, Strides st) {
   constexpr int CH = D / 8;       // 16-byte chunks per row
   constexpr int RG = 256 / CH;    // row groups
   constexpr int RPT = kBlock / RG;  // rows per thread
@@ -97,7 +99,13 @@ __global__ void __launch_bounds__(256) pool_means_kernel(const uint16_t* __restr
       float s = 0.f;
 #pragma unroll
       for (int w8 = 0; w8 < 8; ++w8) s += part[w8][tid];
-      dst[(static_cast<long long>(bh) * NB + j) * D + tid] = s / static_cast<float>(n);
+      const float mean = s / static_cast<float>(n);
+      const long long o = (static_cast<long long>(bh) * NB + j) * D + tid;
+      dst[o] = mean;
+      if (which > 0) {  // bf16 copies of the pooled keys / values (round to nearest even)
+        uint16_t* d16 = which == 1 ? kbar16 : vbar16;
+        d16[o] = static_cast<uint16_t>(__bfloat16_as_ushort(__float2bfloat16_rn(mean)));
+      }
     }
     __syncthreads();
   }
@@ -265,7 +273,8 @@ cudaError_t launch_pool_d(const uint16_t* q, const uint16_t* k, const uint16_t* 
   const int NB = (N + kBlock - 1) / kBlock;
   const long long items = 3ll * BH * NB;
   const int grid1 = static_cast<int>(items < num_sms * 8ll ? items : num_sms * 8ll);
-  pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, BH, H, N, NB, st);
+  pool_means_kernel<D><<<grid1, 256, 0, stream>>>(q, k, v, p.qbar, p.kbar, p.vbar, p.kbar16, p.vbar16, BH, H, N,
+                                                   NB, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int smem = static_cast<int>(sizeof(KeyStatsSmem<D>));

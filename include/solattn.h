@@ -63,6 +63,8 @@ enum solattn_status_code {
  *   qbar, kbar, vbar  [B][H][N_b][d]  block means over valid tokens
  *   kmean             [B][H][d]       mean of the pooled keys (each block counts once)
  *   kcov              [B][H][d][d]    covariance of the pooled keys, divided by N_b
+ *   kbar16, vbar16    [B][H][N_b][d]  kbar and vbar rounded to bf16 (operands of the
+ *                                     per-token correction's MMAs)
  * (paithon.it, "Una soglia per ogni riga", last paragraph: the mean and the
  * d x d second-moment matrix of the pooled keys give every proxy row's mean and
  * spread; solattn_forward evaluates them per query block from kmean and kcov.)
@@ -73,6 +75,8 @@ typedef struct {
   float* vbar;
   float* kmean;
   float* kcov;
+  void* kbar16;
+  void* vbar16;
 } solattn_pooled_t;
 
 /*
@@ -181,14 +185,22 @@ typedef struct {
   float topp;    /* top-p rule: mass fraction (NaN rejected) */
   int n_forced;  /* leading key blocks always kept, >= 0 (0 = none) */
   solattn_strides_t strides;  /* of q, k, v and out; all zero = contiguous [B][H][N][d] */
+  int correction;  /* 0: block-level proxy score s_hat_ij for a skipped block (the
+                      library's definition); 1: per token, s q_t . kbar_j (the
+                      literal reading of "Scegliere mentre si calcola": each token
+                      of a skipped block carries the block's mean key), value
+                      vbar_j either way */
 } solattn_options_t;
 
 /*
  * solattn_forward with the kept-set rule, forced blocks and tensor strides of
  * *opts (host memory, read during the call). solattn_forward(..., beta, ...)
- * equals this call with {SOLATTN_RULE_THRESHOLD, beta, 0, 0, 0, {0, 0, 0}}.
+ * equals this call with {SOLATTN_RULE_THRESHOLD, beta, 0, 0, 0, {0, 0, 0}, 0}.
  * Errors as for solattn_forward, plus SOLATTN_ERR_ARG for a null opts, an
- * unknown rule, a NaN beta/topp, a negative n_forced or invalid strides.
+ * unknown rule, a NaN beta/topp, a negative n_forced, invalid strides or a
+ * correction other than 0 / 1. With correction = 1 the skipped blocks of the
+ * unit's two query blocks are attended as extra 128-key tiles of pooled keys
+ * (kbar16, vbar16), each column weighted by n_j.
  */
 int solattn_forward_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                        const solattn_pooled_t* pooled, const solattn_options_t* opts, void* out,

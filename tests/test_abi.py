@@ -90,6 +90,7 @@ def test_forward_ex_argument_errors(L):
     assert call(O(_lib.RULE_THRESHOLD, math.nan, 0, 0.0, 0)) == _lib.ERR_ARG
     assert call(O(_lib.RULE_TOPP, 0.0, 0, math.nan, 0)) == _lib.ERR_ARG
     assert call(O(_lib.RULE_TOPK, 0.0, 3, 0.0, -1)) == _lib.ERR_ARG        # negative forced count
+    assert call(O(_lib.RULE_THRESHOLD, 0.5, 0, 0.0, 0, _lib.StridesStruct(0, 0, 0), 2)) == _lib.ERR_ARG
     bad = _pooled_struct()
     bad.kcov = None
     assert L.solattn_forward_ex(FAKE, FAKE, FAKE, 1, 1, 128, 64, ctypes.byref(bad),
@@ -129,13 +130,13 @@ def test_pooled_layout_sizes_and_alignment(L):
     assert L.solattn_pooled_layout(B, H, N, d, None, None, ctypes.byref(n)) == 0
     nb = math.ceil(N / 64)
     r = lambda x: (x + 255) // 256 * 256
-    want = 3 * r(B * H * nb * d * 4) + r(B * H * d * 4) + r(B * H * d * d * 4)
+    want = 3 * r(B * H * nb * d * 4) + r(B * H * d * 4) + r(B * H * d * d * 4) + 2 * r(B * H * nb * d * 2)
     assert n.value == want
     st = _lib.PooledStruct()
     base = 0x10000000
     assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base), ctypes.byref(st), None) == 0
     ptrs = [getattr(st, f) for f, _ in _lib.PooledStruct._fields_]
     assert ptrs[0] == base and all(p % 256 == 0 for p in ptrs) and ptrs == sorted(ptrs)
-    assert ptrs[-1] + r(B * H * d * d * 4) == base + want
+    assert ptrs[-1] + r(B * H * nb * d * 2) == base + want
     assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base + 8), ctypes.byref(st), None) == _lib.ERR_ALIGN
     assert L.solattn_pooled_layout(B, H, N, 80, None, None, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED
