@@ -44,9 +44,16 @@ __device__ unsigned long long g_trace[40][4096];
   do {                                                                       \
     if (blockIdx.x == 0 && (idx) < 4096) g_trace[(ev)][(idx)] = clock64();   \
   } while (0)
+#define SOLATTN_TRACE_VALUE(ev, idx, val)                                    \
+  do {                                                                       \
+    if (blockIdx.x == 0 && (idx) < 4096) g_trace[(ev)][(idx)] = (val);       \
+  } while (0)
 #else
 #define SOLATTN_TRACE_EVENT(ev, idx) \
   do {                               \
+  } while (0)
+#define SOLATTN_TRACE_VALUE(ev, idx, val) \
+  do {                                    \
   } while (0)
 #endif
 
@@ -79,7 +86,7 @@ enum : uint32_t {
   kSiteOFull,
   kSiteRouteChunk,
   kSiteQFree,
-  kSiteBDone,
+  kSiteBFree,
   kSiteQFull,
   kSiteMlReady,
   kSitePvDone,
@@ -97,6 +104,14 @@ struct __align__(1024) Smem {
   uint8_t qt[kBM * D * 2];               // Q tile of the unit, SW128 K-major panels of 128 rows
   uint8_t kt[kKStages][kBM * D * 2];     // K tiles, same layout
   uint8_t vt[kVStages][kBN * D * 2];     // V blocks, SW128 panels of 64 rows
+  // Per-token correction: one extra K = 16 step of each pooled tile's QK adds,
+  // for the row's query block g, columns 2g and 2g + 1 of the bias tile to the
+  // score: -1e30 on the key blocks g kept (and on pads), else ln(n_j) sqrt(d)
+  // as a bf16 hi + lo pair. ebias is the constant 0/1 query-side operand. Both are
+  // K-major without swizzle (core matrices 8 rows x 16 B; 128 B between the
+  // two along K, 256 B between groups of 8 rows).
+  uint8_t ebias[kBM * 32];
+  uint8_t kbias[kBM * 32];
   float rchunk[2][kChunk][D];        // routing: pooled keys of a chunk, double-buffered
   float cnum[2][2][D];               // correction numerator per slot and block
   float cden[2][2];
@@ -125,6 +140,7 @@ struct __align__(1024) Smem {
   uint64_t route_full[2], route_empty[2];
   uint64_t rfull[2];                 // routing chunk buffers landed
   uint64_t mma_done[2];
+  uint64_t b_free;                   // per-token correction: the bias tile was read by its QK
   float xm[kBM][2];                  // softmax: row max of each key half (exchange)
   float xl[kBM][2];                  // softmax: row sum of each key half (epilogue)
   uint32_t tmem_base;
@@ -673,6 +689,12 @@ __device__ __forceinline__ void softmax_slice(const uint32_t* x, uint64_t sc2, u
   }
 }
 
+// A bf16 hi + lo pair (hi in the low half) whose sum is w to about 16 bits.
+__device__ __forceinline__ uint32_t bias_pair(float w) {
+  const float hi = __uint_as_float((pack_bf16x2(w, 0.f) & 0xFFFFu) << 16);
+  return pack_bf16x2(hi, w - hi);
+}
+
 // Tiles of a unit: TT of kept blocks (two per tile) and, with the per-token
 // correction, TP of pooled keys (128 per tile, every key block of the head;
 // columns are masked per query block to the blocks it skipped). V blocks: T
@@ -748,6 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.q_free, 1);
     mbar_init(&sm.mma_done[0], 1);
     mbar_init(&sm.mma_done[1], 1);
+    mbar_init(&sm.b_free, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -762,6 +785,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (TOKEN) {
       prefetch_tensormap(&tmKb);
       prefetch_tensormap(&tmVb);
+    }
+  }
+  if constexpr (TOKEN) {
+    if (warp == 12) {
+      // the constant query-side operand: row r of query block g = r / 64 has
+      // ones in columns 2g, 2g + 1; columns 8-15 of both tiles stay zero
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane * 4 + i;
+        constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 ones
+        uint8_t* e = &sm.ebias[(r >> 3) * 256 + (r & 7) * 16];
+        *reinterpret_cast<uint4*>(e) = r < 64 ? make_uint4(kOnes, 0u, 0u, 0u) : make_uint4(0u, kOnes, 0u, 0u);
+        *reinterpret_cast<uint4*>(e + 128) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(&sm.kbias[(r >> 3) * 256 + 128 + (r & 7) * 16]) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
     }
   }
   tc_fence_before();
@@ -810,6 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.unit[s] = u;
         mbar_arrive(&sm.route_full[s]);
         SOLATTN_TRACE_EVENT(14, n);
+        SOLATTN_TRACE_VALUE(19, n, static_cast<unsigned long long>(sm.count[s]));
       }
       // the Q tile is free once every QK of the previous unit has completed
       bool okq = true;
@@ -830,6 +869,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= TMA producers: warp 12 = K tiles, warp 14 = V blocks =======================
     const bool isK = warp == 12;
     uint32_t g = 0;  // K: global tile index; V: global block index
+    uint32_t nbias = 0, wfull = 0, wlast = 0, wmask = 0;  // per-token correction: bias tiles written, entries
+    if constexpr (TOKEN) {
+      // a pooled key stands for the n_j keys of its block: ln(n_j) sqrt(d) in raw score units
+      const float sd = sqrtf(static_cast<float>(D));
+      wfull = bias_pair(logf(static_cast<float>(kBN)) * sd);
+      wlast = bias_pair(logf(static_cast<float>(P.N - (P.NB - 1) * kBN)) * sd);
+      wmask = pack_bf16x2(-1e30f, 0.f);
+    }
     for (int n = 0;; ++n) {
       const int s = n & 1;
       if (!warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullProd, 0)) break;
@@ -855,6 +902,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             jj[0] = 2 * (t - ut.TT);
             jj[1] = jj[0] + 1;
+          }
+          if constexpr (TOKEN) {
+            if (pooled) {
+              // the previous pooled tile's QK has read the bias tile
+              if (nbias >= 1 && !warp_wait(&sm.b_free, (nbias - 1) & 1, abort_flag, st, kSiteBFree, u)) break;
+              ++nbias;
+              const int jb = jj[0] * kBN;  // first pooled key of the tile
+              for (int i = 0; i < 4; ++i) {
+                const int r = lane * 4 + i, j = jb + r;
+                uint32_t w0 = wmask, w1 = wmask;
+                if (j < P.NB) {
+                  const uint32_t w = j == P.NB - 1 ? wlast : wfull;
+                  if (!((sm.bits[s][0][j >> 5] >> (j & 31)) & 1u)) w0 = w;
+                  if (!((sm.bits[s][1][j >> 5] >> (j & 31)) & 1u)) w1 = w;
+                }
+                *reinterpret_cast<uint4*>(&sm.kbias[(r >> 3) * 256 + (r & 7) * 16]) = make_uint4(w0, w1, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
           }
 #ifdef SOLATTN_TEST_HOOKS
           if (gt == 0 && static_cast<int>(blockIdx.x) == g_hook_skip_cta) continue;  // this tile never arrives
@@ -929,6 +996,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t qdesc = sw128_desc(smem_u32(&sm.qt[0]), 16, 1024);
     const uint64_t kdesc0 = sw128_desc(smem_u32(&sm.kt[0][0]), 16, 1024);
     const uint64_t vdesc0 = sw128_desc(smem_u32(&sm.vt[0][0]), 8192, 1024);
+    const uint64_t edesc = nosw_desc(smem_u32(&sm.ebias[0]), 128, 256);
+    const uint64_t bdesc = nosw_desc(smem_u32(&sm.kbias[0]), 128, 256);
     const uint32_t colO = tmem + kColO;
     uint32_t gtile = 0, gblk = 0;
     uint32_t pv_waited = 0;  // QK issuer: tiles whose PV completion it has observed
@@ -964,8 +1033,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t off = (((kk / 4) * kBM * 128) + (kk % 4) * 32) >> 4;
               mma_ss(tmem + slot * 128, qdesc + off, kd + off, idesc, kk > 0 ? 1u : 0u);
             }
+            const bool pooled = TOKEN && t >= ut.TT;
+            if (pooled) mma_ss(tmem + slot * 128, edesc, bdesc, idesc, 1u);  // + the tile's mask and weights
             mma_commit(&sm.s_full[slot]);
             mma_commit(&sm.k_empty[stg]);
+            if (pooled) mma_commit(&sm.b_free);
             if (t == TT - 1) mma_commit(&sm.q_free);
             SOLATTN_TRACE_EVENT(10, gt);
           }
@@ -1026,9 +1098,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nlast = P.N - (P.NB - 1) * kBN;
     constexpr int DH = D / 2;                 // O / output columns owned by this warp
     const uint32_t colO = tmem + kColO + lane_off + hh * DH;
-    // per-token correction: a pooled key stands for n_j tokens, log2(n_j) added
-    // to its score (in raw score units)
-    const float wfull = 6.f / sl2, wlast = __log2f(static_cast<float>(nlast)) / sl2;
     uint32_t gtile = 0;
     for (int n = 0;; ++n) {
       const int s = n & 1;
@@ -1050,8 +1119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool pooled = TOKEN && t >= ut.TT;
         bool kept;
         int nv = kBN;
-        uint64_t use = 0ull;  // pooled tile: this half's columns whose block this row's query block skipped
-        int j0 = 0;
         if (!pooled) {
           uint32_t entry = 0u;
 #pragma unroll
@@ -1062,28 +1129,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           kept = (entry >> (14 + blk)) & 1u;
           nv = ((entry & 0x3FFF) == static_cast<uint32_t>(P.NB - 1)) ? nlast : kBN;
         } else {
-          j0 = 128 * (t - ut.TT) + 64 * hh;  // first pooled key of this half (a multiple of 64)
+          // pooled keys: the half counts while one of its columns is a block the
+          // row's query block skipped (the QK's bias step put -1e30 on the rest)
+          const int j0 = 128 * (t - ut.TT) + 64 * hh;  // first pooled key of this half
+          kept = false;
           if (hh < nb) {
-            const uint64_t kb = static_cast<uint64_t>(sm.bits[s][blk][j0 >> 5]) |
-                                (static_cast<uint64_t>(sm.bits[s][blk][(j0 >> 5) + 1]) << 32);
-            const int valid = min(64, P.NB - j0);
-            use = ~kb & (valid >= 64 ? ~0ull : ((1ull << valid) - 1ull));
+            const int valid = P.NB - j0;  // > 0
+            const uint32_t u0 = ~sm.bits[s][blk][j0 >> 5] & (valid >= 32 ? ~0u : ((1u << valid) - 1u));
+            const uint32_t u1 = valid <= 32 ? 0u
+                                            : ~sm.bits[s][blk][(j0 >> 5) + 1] &
+                                                  (valid >= 64 ? ~0u : ((1u << (valid - 32)) - 1u));
+            kept = (u0 | u1) != 0u;
           }
-          kept = use != 0ull;
         }
         const bool okw = warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
         tc_fence_after();
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(0, gt);
+        if (lane == 0 && warp == 4) SOLATTN_TRACE_EVENT(27, gt);
         uint32_t sv[64];
         if (kept && okw) tmem_ld32x2_wait(colS + 64 * hh, colS + 64 * hh + 32, sv);
-        if (TOKEN && pooled && kept && okw) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float w = (j0 + c == P.NB - 1) ? wlast : wfull;
-            sv[c] = ((use >> c) & 1ull) ? __float_as_uint(__uint_as_float(sv[c]) + w) : 0xFF800000u;
-          }
-        }
+        if (lane == 0 && (warp & 3) == 0) SOLATTN_TRACE_EVENT(warp == 0 ? 5 : 25, gt);
         const float mx = (kept && okw) ? tile_max(sv, nv) * sl2 : -INFINITY;
+        if (lane == 0 && (warp & 3) == 0) SOLATTN_TRACE_EVENT(warp == 0 ? 6 : 26, gt);
         // Does a row of this group need a new reference max (or did a wait fail)?
         // The barrier also orders this group's S reads before the other half's
         // P stores into the same columns.

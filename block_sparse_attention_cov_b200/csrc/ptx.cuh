@@ -347,6 +347,22 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand without swizzle: 8-row x
+// 16-byte core matrices, lbo_bytes between core matrices along K, sbo_bytes
+// between groups of 8 rows.
+__device__ __forceinline__ uint64_t nosw_desc(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;  // layout type 0 (no swizzle) at bits 61-63
+  return d;
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to the
+// async proxy (tensor-core operand reads) once a later barrier orders them.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // D format F32 = 1 at bits [4,6); A format BF16 = 1 at [7,10); B format BF16 = 1
 // at [10,13); A major at bit 15, B major at bit 16 (0 = K-major, 1 = MN-major);
