@@ -564,20 +564,26 @@ struct KeyWalk {
   const uint32_t* b0;
   const uint32_t* b1;
   int w, pos;
-  uint32_t rem;
-  __device__ __forceinline__ KeyWalk(const uint32_t* x0, const uint32_t* x1) : b0(x0), b1(x1), w(-1), pos(0), rem(0u) {}
+  uint32_t rem, c0, c1;  // unvisited bits of word w, and the word itself (both bitmaps)
+  __device__ __forceinline__ KeyWalk(const uint32_t* x0, const uint32_t* x1)
+      : b0(x0), b1(x1), w(-1), pos(0), rem(0u), c0(0u), c1(0u) {}
   __device__ __forceinline__ uint32_t next() {
     if constexpr (!ROUTE) {
       return static_cast<uint32_t>(pos++) | 0xC000u;
     } else {
+      // shared memory is read only when the walk moves to the next word: the
+      // callers sit between barriers and fences, so nothing read here would
+      // stay in registers across calls otherwise
       while (rem == 0u) {
         if (w + 1 >= kNbMax / 32) return 0u;
         ++w;
-        rem = b0[w] | b1[w];
+        c0 = b0[w];
+        c1 = b1[w];
+        rem = c0 | c1;
       }
       const int bit = __ffs(rem) - 1;
       rem &= rem - 1u;
-      const uint32_t f = ((b0[w] >> bit) & 1u) | (((b1[w] >> bit) & 1u) << 1);
+      const uint32_t f = ((c0 >> bit) & 1u) | (((c1 >> bit) & 1u) << 1);
       return static_cast<uint32_t>(w * 32 + bit) | (f << 14);
     }
   }
@@ -1142,7 +1148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             kept = (u0 | u1) != 0u;
           }
         }
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(7, gt);
         const bool okw = warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(8, gt);
         tc_fence_after();
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(0, gt);
         if (lane == 0 && warp == 4) SOLATTN_TRACE_EVENT(27, gt);

@@ -107,9 +107,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Waits for the phase of `bar` with the given parity to complete. Returns false
 // (after recording an error in `st` and raising the CTA-wide abort flag) when
 // the wait takes longer than the budget or another role has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          DeviceStatus* st, uint32_t site, uint32_t unit) {
-  if (mbar_test(bar, parity)) return true;  // already complete: no suspend
+// The slow path lives out of line so that the hot loops calling mbar_wait
+// carry only the phase test (smaller code, fewer instruction-cache misses).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                   DeviceStatus* st, uint32_t site, uint32_t unit) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -127,6 +128,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          DeviceStatus* st, uint32_t site, uint32_t unit) {
+  if (mbar_test(bar, parity)) return true;  // already complete: no suspend
+  return mbar_wait_slow(bar, parity, abort_flag, st, site, unit);
 }
 
 // Wait used during teardown: bounded, records nothing.
