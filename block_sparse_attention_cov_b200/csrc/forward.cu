@@ -90,6 +90,7 @@ enum : uint32_t {
   kSiteQFull,
   kSiteMlReady,
   kSitePvDone,
+  kSiteEFull,
 };
 
 template <int D, bool SEL = false>
@@ -141,6 +142,11 @@ struct __align__(1024) Smem {
   uint64_t rfull[2];                 // routing chunk buffers landed
   uint64_t mma_done[2];
   uint64_t b_free;                   // per-token correction: the bias tile was read by its QK
+  // Key-list entries of the key tiles (both halves), published by the K
+  // producer, which walks the list anyway, for the softmax warps: a ring of 8
+  // tiles, one barrier per slot
+  uint32_t kentry[8][2];
+  uint64_t e_full[8];
   float xm[kBM][2];                  // softmax: row max of each key half (exchange)
   float xl[kBM][2];                  // softmax: row sum of each key half (epilogue)
   uint32_t tmem_base;
@@ -777,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.mma_done[0], 1);
     mbar_init(&sm.mma_done[1], 1);
     mbar_init(&sm.b_free, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&sm.e_full[i], 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -874,7 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 12 || warp == 14) {
     // ======================= TMA producers: warp 12 = K tiles, warp 14 = V blocks =======================
     const bool isK = warp == 12;
-    uint32_t g = 0;  // K: global tile index; V: global block index
+    uint32_t g = 0;   // K: global tile index; V: global block index
+    uint32_t gk = 0;  // K: key tiles published (entry ring position)
     uint32_t nbias = 0, wfull = 0, wlast = 0, wmask = 0;  // per-token correction: bias tiles written, entries
     if constexpr (TOKEN) {
       // a pooled key stands for the n_j keys of its block: ln(n_j) sqrt(d) in raw score units
@@ -903,8 +911,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool pooled = TOKEN && t >= ut.TT;  // a tile of pooled keys (per-token correction)
           int jj[2];
           if (!pooled) {
-            jj[0] = walk.next() & 0x3FFF;
-            jj[1] = nb == 2 ? (walk.next() & 0x3FFF) : 0;
+            const uint32_t e0 = walk.next(), e1 = nb == 2 ? walk.next() : 0u;
+            jj[0] = e0 & 0x3FFF;
+            jj[1] = e1 & 0x3FFF;
+            // Publish the tile's entries for the softmax warps. Slot reuse is
+            // safe: this tile's stage was released by QK(t - KS), so the softmax
+            // has finished tile t - KS - 3 and is past every older slot user.
+            const uint32_t ek = gk++;
+            if (elect_one()) {
+              sm.kentry[ek & 7][0] = e0;
+              sm.kentry[ek & 7][1] = e1;
+              mbar_arrive(&sm.e_full[ek & 7]);
+            }
+            __syncwarp();
           } else {
             jj[0] = 2 * (t - ut.TT);
             jj[1] = jj[0] + 1;
@@ -1104,7 +1123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nlast = P.N - (P.NB - 1) * kBN;
     constexpr int DH = D / 2;                 // O / output columns owned by this warp
     const uint32_t colO = tmem + kColO + lane_off + hh * DH;
-    uint32_t gtile = 0;
+    uint32_t gtile = 0, gkey = 0;  // tiles / key tiles consumed so far
     for (int n = 0;; ++n) {
       const int s = n & 1;
       bool okr = warp_wait(&sm.route_full[s], (n >> 1) & 1, abort_flag, st, kSiteRouteFullSoft, 0);
@@ -1117,21 +1136,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int TT = ut.total();
       float m = -INFINITY, l = 0.f;  // m: the row's shared reference max; l: this half's sum
       bool ok = true;
-      KeyWalk<ROUTE> walk(sm.bits[s][0], sm.bits[s][1]);
       for (int t = 0; t < TT; ++t) {
         const uint32_t gt = gtile + t, slot = gt % 3;
+        if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(9, gt);
         const uint32_t colS = tmem + slot * 128 + lane_off;
         const int nb = ut.halves(t, P.NB);
         const bool pooled = TOKEN && t >= ut.TT;
         bool kept;
         int nv = kBN;
+        bool oke = true;
         if (!pooled) {
-          uint32_t entry = 0u;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t e = h < nb ? walk.next() : 0u;
-            if (h == hh) entry = e;
-          }
+          // this half's key-list entry, published by the K producer
+          const uint32_t ek = gkey++;
+          oke = warp_wait(&sm.e_full[ek & 7], (ek >> 3) & 1, abort_flag, st, kSiteEFull, u);
+          const uint32_t entry = hh < nb ? sm.kentry[ek & 7][hh] : 0u;
           kept = (entry >> (14 + blk)) & 1u;
           nv = ((entry & 0x3FFF) == static_cast<uint32_t>(P.NB - 1)) ? nlast : kBN;
         } else {
@@ -1149,7 +1167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(7, gt);
-        const bool okw = warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
+        const bool okw = oke && warp_wait(&sm.s_full[slot], (gt / 3) & 1, abort_flag, st, kSiteSFull, u);
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(8, gt);
         tc_fence_after();
         if (lane == 0 && warp == 0) SOLATTN_TRACE_EVENT(0, gt);
