@@ -188,13 +188,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// Routing (warps 4-7, 128 threads): the pooled keys and values of the head are
-// streamed through shared memory in chunks of 32 key blocks (bulk async copies,
-// double-buffered). Per chunk: every warp scores 8 key blocks against both
-// query blocks of the unit (one float4 column slice per lane, transposed
-// butterfly reduction), the threshold test sets the kept bits, and the skipped
-// blocks' weights n_j e^{s_hat - M} are folded into per-column correction sums
-// (one column per thread). The proxy row never leaves shared memory.
+// Routing (warps 8-11, 128 threads): the pooled keys of the head are streamed
+// through shared memory in chunks of 16 key blocks (bulk async copies,
+// double-buffered); the pooled values go from L2 to registers. Per chunk:
+// every warp scores 4 key blocks against both query blocks of the unit (one
+// float4 column slice per lane, transposed butterfly reduction), the rule sets
+// the kept bits, and the skipped blocks' weights n_j e^{s_hat - M} are folded
+// into per-column correction sums (one column per thread); no proxy map in HBM.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -204,7 +204,7 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
-// Returns false if a bounded wait gave up (the CTA is aborting).
+// Helpers of the routing warps and of the top-k / top-p cut.
 // Order-preserving map of a float to an unsigned key (x < y <=> key(x) < key(y)).
 __device__ __forceinline__ uint32_t order_key(float x) {
   const uint32_t u = __float_as_uint(x);
@@ -217,10 +217,10 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// RULE 0: per-row threshold tau_i = mu_i + beta sigma_i, decided chunk by
-// chunk as the scores are produced. RULE 1 / 2 (top-k / top-p): a first pass
-// stores the unit's two proxy rows, each row's cut is found by bisection on
-// the order keys, and a second pass decides and folds the corrections.
+// RULE 0: per-row threshold tau_i = mu_i + beta sigma_i, decided chunk by chunk
+// as the scores are produced. RULE 1 / 2 (top-k / top-p): a first pass stores
+// the unit's two proxy rows, a bisection on the order keys finds each row's cut,
+// and a second pass decides and folds. False if a bounded wait gave up.
 template <int D, int RULE>
 __device__ bool route_unit(Smem<D, RULE != 0>& sm, const Params& P, int s, int bh, int pair, int rt, uint32_t& chunk_ctr,
                            volatile int* abort_flag, DeviceStatus* st, int u) {
