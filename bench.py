@@ -1,7 +1,7 @@
 """Benchmark of the Sol-Attn forward (pool + fused forward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload wan_75k] [--beta B]
+                    [--workload wan_75k] [--beta B | --density D]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 solattn_pool (block means, key mean and covariance) followed by
@@ -229,7 +229,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
-    beta = args.beta if args.beta is not None else load_beta(args.workload)[0]
+    beta = args.beta if args.beta is not None else load_beta(args.workload, args.density)[0]
     q, k, v = make_qkv(wl, 0, heads=[(0, 0)])
     times, flops = [], 0.0
     for step in range(args.warmup + args.steps):
@@ -263,7 +263,7 @@ def run_ours(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload]
     if args.heads:
         wl = dataclasses.replace(wl, H=args.heads)
-    beta = args.beta if args.beta is not None else load_beta(args.workload)[0]
+    beta = args.beta if args.beta is not None else load_beta(args.workload, args.density)[0]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
     peaks = load_peaks()
 
@@ -460,6 +460,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan_75k", choices=sorted(WORKLOADS))
     ap.add_argument("--beta", type=float, default=None)
+    ap.add_argument("--density", type=float, default=None,
+                    help="use the calibrated beta of this mean kept-block density (e.g. 0.05 on the sweeps)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--cpu-blocks", type=int, default=600)
     ap.add_argument("--rule", choices=["threshold", "topk", "topp"], default="threshold",
