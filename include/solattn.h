@@ -12,11 +12,12 @@
  * N_b = ceil(N / 64), n_j = valid tokens of block j (64, or fewer for the last),
  * s = 1/sqrt(d).
  *
- * Layouts (row-major, contiguous, no padding):
+ * Layouts (row-major; contiguous unless solattn_pool_ex / solattn_forward_ex
+ * are given other strides):
  *   q, k, v, out        bf16 [B][H][N][d]   (passed as raw 16-bit words)
  *   lse                 fp32 [B][H][N]      natural log of the softmax sum
  *   density_out         int32 [B][H][N_b]   |S_i| = kept key blocks per query block
- *   pooled buffers      fp32, see solattn_pooled_t
+ *   pooled buffers      fp32 (plus bf16 copies of kbar, vbar), see solattn_pooled_t
  *
  * Ownership: the caller allocates every buffer, on the device unless a function
  * says otherwise. No call allocates device memory. Nothing is retained after a
