@@ -169,10 +169,18 @@ def forward(q, k, v, stats: PooledStats, beta: float = 0.0, out=None, lse=None, 
 
 
 def dense(q, k, v, out=None, lse=None, ws=None, want_lse: bool = True):
-    """Dense attention through the same kernel with routing off (solattn_dense)."""
+    """Dense attention through the same kernel with routing off (solattn_dense).
+    solattn_dense takes no strides: q, k, v and out must be contiguous
+    [B, H, N, d] (a permuted, sliced or expanded view is rejected, since the
+    kernel would read it as contiguous memory)."""
+    for t in (q, k, v) + (() if out is None else (out,)):
+        if not t.is_contiguous():
+            raise ValueError("dense() needs contiguous [B, H, N, d] q, k, v and out")
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     out = torch.empty_like(q) if out is None else out
+    if out.shape != q.shape or out.dtype != torch.bfloat16:
+        raise ValueError("out must be a bf16 tensor of q's shape")
     if lse is None and want_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     ws = workspace(q.device) if ws is None else ws

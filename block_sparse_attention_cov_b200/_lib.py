@@ -18,6 +18,7 @@ EXPORTS = (
     "solattn_forward_noalloc",
     "solattn_forward_ex",
     "solattn_pool_ex",
+    "solattn_noalloc_status",
 )
 
 OK = 0
@@ -58,16 +59,9 @@ class OptionsStruct(ctypes.Structure):
 _lib = None
 
 
-def lib() -> ctypes.CDLL:
-    """The loaded library. Raises if it has not been built: there is no fallback."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(
-            f"{LIB_PATH} is missing; build it with `python -m block_sparse_attention_cov_b200.build`"
-        )
-    L = ctypes.CDLL(LIB_PATH)
+def declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Sets the argument and result types of every exported call on a loaded
+    copy of the library (the product build or its test-hook variant)."""
     i, vp, f, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
     L.solattn_pooled_layout.argtypes = [i, i, i, i, vp, ctypes.POINTER(PooledStruct), ctypes.POINTER(sz)]
     L.solattn_pooled_layout.restype = i
@@ -83,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.solattn_strerror.restype = ctypes.c_char_p
     L.solattn_forward_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
     L.solattn_forward_noalloc.restype = i
+    L.solattn_noalloc_status.argtypes = [vp]
+    L.solattn_noalloc_status.restype = i
     L.solattn_forward_ex.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(PooledStruct),
                                      ctypes.POINTER(OptionsStruct), vp, vp, vp, vp, sz, vp]
     L.solattn_forward_ex.restype = i
@@ -91,8 +87,20 @@ def lib() -> ctypes.CDLL:
     L.solattn_pool_ex.restype = i
     L.solattn_version.argtypes = []
     L.solattn_version.restype = i
-    _lib = L
     return L
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library. Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing; build it with `python -m block_sparse_attention_cov_b200.build`"
+        )
+    _lib = declare(ctypes.CDLL(LIB_PATH))
+    return _lib
 
 
 def strerror(code: int) -> str:

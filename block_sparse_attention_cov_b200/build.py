@@ -18,7 +18,7 @@ LIB = os.path.join(PKG, "libsolattn.so")
 # makes one CTA skip its first K tile and shortens the bounded-wait budget.
 LIB_HOOKS = os.path.join(PKG, "libsolattn_testhooks.so")
 SOURCES = ["api.cu", "pool.cu", "forward.cu"]
-HEADERS = ["kernels.h", "ptx.cuh"]
+HEADERS = ["kernels.h", "ptx.cuh", "fwd_common.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/solattn.h: argument checks, buffer
 // layout helpers and stream-ordered launches. No allocation happens here.
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -17,8 +18,10 @@ using solattn::PooledPtrs;
 static_assert(sizeof(DeviceStatus) <= SOLATTN_WORKSPACE_BYTES, "workspace too small for the status block");
 
 constexpr int kMaxDevices = 64;
-int g_sms[kMaxDevices];   // 0 = not yet queried, -1 = not an sm_100 device
-int g_cc[kMaxDevices];
+// Multiprocessor count per device: 0 = not yet queried, -1 = not an sm_100
+// device. Filled lazily; concurrent first calls may both query the device and
+// store the same value, which the atomic makes well defined.
+std::atomic<int> g_sms[kMaxDevices];
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -54,29 +57,33 @@ int current_device_sms(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SOLATTN_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SOLATTN_ERR_DEVICE;
-  if (g_sms[dev] == 0) {
+  int n = g_sms[dev].load(std::memory_order_acquire);
+  if (n == 0) {
     int major = 0, minor = 0, count = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return SOLATTN_ERR_CUDA;
-    g_cc[dev] = major * 10 + minor;
-    g_sms[dev] = (major == 10 && minor == 0) ? count : -1;
+    n = (major == 10 && minor == 0) ? count : -1;
+    g_sms[dev].store(n, std::memory_order_release);
   }
-  if (g_sms[dev] < 0) return SOLATTN_ERR_DEVICE;
-  *sms = g_sms[dev];
+  if (n < 0) return SOLATTN_ERR_DEVICE;
+  *sms = n;
   return SOLATTN_OK;
 }
 
 // Strides of q, k, v, out: all zero means contiguous [B][H][N][d]; otherwise
-// every stride a multiple of 8 elements (16 bytes: 128-bit loads, TMA) and the
-// token stride at least d.
-int resolve_strides(const solattn_strides_t* in, int H, int N, int d, solattn::Strides* out) {
+// every stride a multiple of 8 elements (16 bytes: 128-bit loads, TMA), the
+// token stride at least d, and the head (batch) stride non-zero when there is
+// more than one head (batch): out shares these strides, and two heads writing
+// the same rows would race.
+int resolve_strides(const solattn_strides_t* in, int B, int H, int N, int d, solattn::Strides* out) {
   if (!in || (in->batch == 0 && in->head == 0 && in->token == 0)) {
     *out = solattn::Strides{static_cast<long long>(H) * N * d, static_cast<long long>(N) * d, d};
     return SOLATTN_OK;
   }
   if (in->batch < 0 || in->head < 0 || in->token < d) return SOLATTN_ERR_ARG;
+  if ((H > 1 && in->head == 0) || (B > 1 && in->batch == 0)) return SOLATTN_ERR_ARG;
   if ((in->batch | in->head | in->token) & 7) return SOLATTN_ERR_ARG;
   *out = solattn::Strides{in->batch, in->head, in->token};
   return SOLATTN_OK;
@@ -98,7 +105,7 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (!aligned16(out)) return SOLATTN_ERR_ALIGN;
   if ((lse && !aligned4(lse)) || (density && !aligned4(density))) return SOLATTN_ERR_ALIGN;
   solattn::Strides strides;
-  if ((rc = resolve_strides(&opt.strides, H, N, d, &strides))) return rc;
+  if ((rc = resolve_strides(&opt.strides, B, H, N, d, &strides))) return rc;
   if (route) {
     if (std::isnan(beta) || std::isnan(opt.topp) || opt.n_forced < 0) return SOLATTN_ERR_ARG;
     if (opt.rule != SOLATTN_RULE_THRESHOLD && opt.rule != SOLATTN_RULE_TOPK && opt.rule != SOLATTN_RULE_TOPP)
@@ -201,7 +208,7 @@ int solattn_pool_ex(const void* q, const void* k, const void* v, int B, int H, i
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
   solattn::Strides st;
-  if ((rc = resolve_strides(strides, H, N, d, &st))) return rc;
+  if ((rc = resolve_strides(strides, B, H, N, d, &st))) return rc;
   if ((rc = check_qkv(q, k, v))) return rc;
   if ((rc = check_pooled(pooled))) return rc;
   int sms = 0;
@@ -235,6 +242,23 @@ int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int
   return run_forward(q, k, v, B, H, N, d, nullptr, opt, false, out, lse, nullptr, workspace, workspace_bytes,
                      stream);
 }
+
+#ifdef SOLATTN_TEST_HOOKS
+// Test builds only (libsolattn_testhooks.so; not declared in include/solattn.h):
+// CTA `skip_cta` never requests its first K tile (-1: none) and every bounded
+// wait gives up after `wait_budget_ns`.
+int solattn_test_set_hook(int skip_cta, unsigned long long wait_budget_ns) {
+  return solattn::set_test_hooks_fwd(skip_cta, wait_budget_ns) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+}
+
+// Test builds only: every later forward copies its units' kept bitmaps to `mask`
+// ([B*H][N_b][ceil(N_b / 32)] uint32, bit j % 32 of word j / 32 = key block j
+// kept) and mu_i, sigma_i, tau_i to `stats` ([B*H][N_b][3] float; NaN where the
+// rule does not define them). NULL, NULL switches the copy off.
+int solattn_test_set_route_dump(uint32_t* mask, float* stats) {
+  return solattn::set_route_dump_fwd(mask, stats) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+}
+#endif
 
 int solattn_status(const void* workspace, void* stream) {
   if (!workspace) return SOLATTN_ERR_WORKSPACE;
@@ -297,6 +321,15 @@ int solattn_forward_noalloc(const void* q, const void* k, const void* v, int B, 
   if ((rc = solattn_pool(q, k, v, B, H, N, d, &pooled, stream))) return rc;
   return solattn_forward(q, k, v, B, H, N, d, &pooled, beta, out, lse, density_out, scratch,
                          SOLATTN_WORKSPACE_BYTES, stream);
+}
+
+int solattn_noalloc_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  DeviceStatus h{};
+  // the status block sits at the start of the static array; a copy from the
+  // symbol allocates nothing
+  if (cudaMemcpyFromSymbol(&h, g_noalloc_scratch, sizeof(h)) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  return h.error == 0 ? SOLATTN_OK : static_cast<int>(h.error);
 }
 
 }  // extern "C"

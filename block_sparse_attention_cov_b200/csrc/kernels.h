@@ -47,4 +47,10 @@ cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream);
 
+#ifdef SOLATTN_TEST_HOOKS
+// Test builds only: hook variables of each kernel's translation unit.
+cudaError_t set_test_hooks_fwd(int skip_cta, unsigned long long wait_budget_ns);
+cudaError_t set_route_dump_fwd(uint32_t* mask, float* stats);
+#endif
+
 }  // namespace solattn

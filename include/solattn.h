@@ -109,8 +109,9 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
  * starts at b * batch + h * head + n * token elements from the base pointer and
  * its d elements are contiguous. {H*N*d, N*d, d} is [B][H][N][d]; {N*H*d, d,
  * H*d} is [B][N][H][d]. Every stride must be a multiple of 8 elements (16
- * bytes) and token >= d; all zero means contiguous [B][H][N][d]. The four
- * tensors share one set of strides.
+ * bytes), token >= d, head != 0 when H > 1 and batch != 0 when B > 1 (out
+ * shares the strides: two heads must not write the same rows); all zero means
+ * contiguous [B][H][N][d]. The four tensors share one set of strides.
  */
 typedef struct {
   long long batch;
@@ -245,13 +246,23 @@ int solattn_status(const void* workspace, void* stream);
  * any stream capture. All calls share the one array and it keeps the last
  * call's contents: calls that overlap on the GPU (other streams, other host
  * threads) race and must be serialised by the caller. The scheduler counter and
- * status word at the start of the array are cleared by every call; the status
- * word is not exposed (a bounded device wait that expires still ends the kernel
- * early instead of hanging, but this call cannot report it).
+ * status word at the start of the array are cleared by every call; a bounded
+ * device wait that expires ends the kernel early (instead of hanging) and is
+ * reported by solattn_noalloc_status, not by this call's return code.
  */
 #define SOLATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
 int solattn_forward_noalloc(const void* q, const void* k, const void* v, int B, int H, int N, int d, float beta,
                             void* out, float* lse, int32_t* density_out, void* stream);
+
+/*
+ * Device status of the last solattn_forward_noalloc call on the current device
+ * (no counterpart on the pages): synchronises `stream`, then copies the status
+ * block out of the static array (no allocation) and returns SOLATTN_OK or
+ * SOLATTN_ERR_TIMEOUT (a bounded wait gave up; that call's outputs are
+ * invalid); SOLATTN_ERR_CUDA if the synchronisation or the copy fails. Calls on
+ * other streams that overlap the one being checked race on the same block.
+ */
+int solattn_noalloc_status(void* stream);
 
 /* Static description of a status code. */
 const char* solattn_strerror(int code);

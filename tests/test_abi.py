@@ -140,3 +140,38 @@ def test_pooled_layout_sizes_and_alignment(L):
     assert ptrs[-1] + r(B * H * nb * d * 2) == base + want
     assert L.solattn_pooled_layout(B, H, N, d, ctypes.c_void_p(base + 8), ctypes.byref(st), None) == _lib.ERR_ALIGN
     assert L.solattn_pooled_layout(B, H, N, 80, None, None, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED
+
+
+def test_noalloc_path_names_no_allocating_call():
+    """The allocation-free entry point and its helpers call no device
+    allocator (checked on the source of the noalloc section of api.cu)."""
+    src = open(os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", "api.cu")).read()
+    section = src[src.index("Allocation-free forward"):]
+    code = re.sub(r"//[^\n]*", "", section)
+    for name in ("cudaMalloc", "cudaMallocAsync", "cudaMallocManaged", "cudaFree", "malloc(", "new ", "torch"):
+        assert name not in code, name
+
+
+def test_strides_reject_aliasing_heads_and_batches(L):
+    """out shares q's strides: a zero head (batch) stride with several heads
+    (batches) would make them write the same rows."""
+    def call(B, H, strides):
+        opts = _lib.OptionsStruct(_lib.RULE_THRESHOLD, 0.5, 0, 0.0, 0, _lib.StridesStruct(*strides), 0)
+        return L.solattn_forward_ex(FAKE, FAKE, FAKE, B, H, 128, 64, ctypes.byref(_pooled_struct()),
+                                    ctypes.byref(opts), FAKE, None, None, None, 0, None)
+
+    assert call(1, 2, (0, 0, 64)) == _lib.ERR_ARG
+    assert call(2, 1, (0, 64, 64)) == _lib.ERR_ARG
+    # one head and one batch: a zero stride there is harmless; the call then
+    # fails later, on the missing workspace
+    assert call(1, 1, (0, 0, 64)) == _lib.ERR_WORKSPACE
+
+
+def test_dense_rejects_non_contiguous_views():
+    import torch
+
+    import block_sparse_attention_cov_b200 as sa
+
+    x = torch.zeros((1, 4, 2, 64), dtype=torch.bfloat16).permute(0, 2, 1, 3)  # [B, N, H, d] seen as [B, H, N, d]
+    with pytest.raises(ValueError, match="contiguous"):
+        sa.dense(x, x, x)

@@ -1,0 +1,161 @@
+"""Kept-set parity, element by element: the kept bitmaps the fused kernel's
+routing warps used, and their mu_i, sigma_i, tau_i, against the oracle's, on
+every workload of the parity suite.
+
+The pages define the kept set of query block i as S_i = {j : s_hat_ij > tau_i}
+with tau_i = mu_i + beta sigma_i (paithon.it, "Una soglia per ogni riga", the
+displayed equation) and state that choosing blocks while the scores are
+produced selects the same set as thresholding the whole row offline
+("Scegliere mentre si calcola"). Acceptance: every (b, h, i, j) decision equals
+the oracle's, except where the fp64 proxy score lies within 1e-4 of tau_i
+(near ties, counted and reported); tau_i, mu_i and sigma_i (fp32 on the GPU)
+within rtol 1e-5 / atol 1e-5 of the fp64 oracle; the kernel's density_out
+equals the popcount of its own bitmap rows.
+
+The bitmaps come from the test-hook build (libsolattn_testhooks.so), whose
+routing warps also copy them out; the product library computes the same kernel
+without the copy.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_cov_b200.inputs import WORKLOADS, Workload, make_qkv
+from hooklib import forward_with_routing
+from oracle import solattn_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+TIE = 1e-4
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "calibrated_beta.json")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _wl(B, H, d, N):
+    return Workload(f"r{B}x{H}x{N}x{d}", B, H, d, (1, 1, N))
+
+
+def _calibrated(name):
+    with open(GOLDEN) as f:
+        return {float(t): v["beta"] for t, v in json.load(f)[name]["targets"].items()}
+
+
+def _check_threshold(q, k, beta, mask, stats, dens, what):
+    """Returns (decisions compared, near ties, flipped near ties)."""
+    B, H = q.shape[:2]
+    n_cmp = n_tie = n_flip = 0
+    for b in range(B):
+        for h in range(H):
+            r = orc.route(q[b, h].double().numpy(), k[b, h].double().numpy(), beta)
+            near = np.abs(r["shat"] - r["tau"][:, None]) <= TIE
+            diff = mask[b, h] != r["mask"]
+            assert not (diff & ~near).any(), (what, b, h, np.argwhere(diff & ~near)[:5])
+            n_cmp += diff.size
+            n_tie += int(near.sum())
+            n_flip += int(diff.sum())
+            assert (dens[b, h] == mask[b, h].sum(-1)).all(), "density_out differs from the kernel's own bitmap"
+            tau = stats[b, h, :, 2].astype(np.float64)
+            fin = np.isfinite(r["tau"])
+            assert (np.isinf(tau) == ~fin).all() and (np.sign(tau[~fin]) == np.sign(r["tau"][~fin])).all()
+            np.testing.assert_allclose(tau[fin], r["tau"][fin], rtol=1e-5, atol=1e-5, err_msg=what)
+            if math.isfinite(beta):
+                np.testing.assert_allclose(stats[b, h, :, 0], r["mu"], rtol=1e-5, atol=1e-5, err_msg=what)
+                np.testing.assert_allclose(stats[b, h, :, 1], r["sigma"], rtol=1e-5, atol=1e-5, err_msg=what)
+    print(f"{what}: {n_cmp} decisions, {n_tie} near ties (|s_hat - tau| <= {TIE}), {n_flip} flipped")
+    return n_cmp, n_tie, n_flip
+
+
+CASES = [
+    ("tiny", WORKLOADS["tiny"], [-math.inf, 0.5, 1.0]),
+    ("mid", WORKLOADS["mid"], [0.0, 0.5, 1.0, 1.5]),
+    ("ragged_d128_b2h3", _wl(2, 3, 128, 1000), [-math.inf, 0.0, 0.7, math.inf]),
+    ("ragged_d64", _wl(1, 2, 64, 64 * 5 + 20), [0.3, math.inf]),
+    ("odd_blocks", _wl(1, 2, 128, 64 * 3), [0.0, -math.inf]),
+    ("single_partial_block", _wl(1, 1, 64, 37), [-math.inf, 0.0, math.inf]),
+]
+
+
+@pytest.mark.parametrize("name,wl,betas", CASES, ids=[c[0] for c in CASES])
+def test_kept_mask_and_tau_match_oracle(name, wl, betas):
+    q, k, v = make_qkv(wl, seed=2)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    for beta in betas:
+        _, _, dens, mask, stats = forward_with_routing(qd, kd, vd, beta)
+        _check_threshold(q, k, beta, mask, stats, dens.cpu().numpy(), f"{name} beta={beta}")
+
+
+@pytest.mark.parametrize("name,heads", [("wan_75k", list(range(40))), ("hunyuan_119k", [0, 23]),
+                                        ("sweep_16k", [0, 13]), ("sweep_32k", [5]), ("sweep_64k", [7]),
+                                        ("sweep_128k", [11])])
+def test_kept_mask_on_the_large_workloads(name, heads):
+    """Every block of the given heads at each calibrated beta of the workload
+    (Wan-like: all 40 heads at the benchmark's 15 % beta)."""
+    wl = WORKLOADS[name]
+    q, k, v = make_qkv(wl, seed=0, heads=[(0, h) for h in heads])
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    for target, beta in sorted(_calibrated(name).items()):
+        _, _, dens, mask, stats = forward_with_routing(qd, kd, vd, beta)
+        _check_threshold(q, k, beta, mask, stats, dens.cpu().numpy(), f"{name} {target:.0%} beta={beta:.4f}")
+        del mask
+
+
+def _rule_near(r, rule, param, N):
+    """Per (i, j): True where the oracle's decision is a near tie at the rule's
+    cut (top-k: a score within 1e-4 of the k-th largest; top-p: the whole row
+    when its cumulative mass crosses p within 1e-4 of the total or the cut
+    value is tied)."""
+    shat = r["shat"]
+    nb = shat.shape[1]
+    near = np.zeros(shat.shape, bool)
+    if rule == "topk" and 0 < param < nb:
+        kth = -np.sort(-shat, axis=1)[:, int(param) - 1]
+        near = np.abs(shat - kth[:, None]) <= TIE
+    elif rule == "topp" and 0.0 < param < 1.0:
+        n = orc.block_counts(N).astype(np.float64)
+        for i in range(nb):
+            order = np.argsort(-shat[i], kind="stable")
+            w = n[order] * np.exp(shat[i, order] - shat[i, order[0]])
+            cum = np.cumsum(w) - param * w.sum()
+            kp = min(int(np.searchsorted(cum, 0.0, side="left")), nb - 1)
+            vstar = shat[i, order[kp]]
+            if (np.abs(cum) <= TIE * w.sum()).any():
+                near[i] = True
+            near[i] |= np.abs(shat[i] - vstar) <= TIE
+    elif rule == "threshold":
+        near = np.abs(shat - r["tau"][:, None]) <= TIE
+    return near
+
+
+@pytest.mark.parametrize("rule,param,n_forced", [("topk", 5, 0), ("topk", 19, 0), ("topp", 0.3, 0),
+                                                 ("topp", 0.9, 0), ("threshold", 1.0, 3), ("topk", 4, 5),
+                                                 ("topp", 0.5, 1)])
+def test_kept_mask_other_rules_and_forced_blocks(rule, param, n_forced):
+    wl = Workload("mid2", 1, 2, 128, (8, 32, 32))
+    q, k, v = make_qkv(wl, seed=23)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    kw = {"topk": int(param)} if rule == "topk" else ({"topp": float(param)} if rule == "topp" else {})
+    beta = param if rule == "threshold" else 0.0
+    _, _, dens, mask, _ = forward_with_routing(qd, kd, vd, beta, rule=rule, n_forced=n_forced, **kw)
+    dens = dens.cpu().numpy()
+    n_tie = n_flip = 0
+    for h in range(wl.H):
+        r = orc.route_rule(q[0, h].double().numpy(), k[0, h].double().numpy(), rule, param, n_forced)
+        near = _rule_near(r, rule, param, wl.N)
+        if n_forced:
+            assert mask[0, h][:, :n_forced].all()
+            near[:, :n_forced] = False
+        diff = mask[0, h] != r["mask"]
+        assert not (diff & ~near).any(), (rule, param, np.argwhere(diff & ~near)[:5])
+        assert (dens[0, h] == mask[0, h].sum(-1)).all()
+        n_tie += int(near.sum())
+        n_flip += int(diff.sum())
+    print(f"{rule}({param}) forced={n_forced}: {n_tie} near ties, {n_flip} flipped")

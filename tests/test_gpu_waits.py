@@ -17,8 +17,8 @@ import pytest
 import torch
 
 from block_sparse_attention_cov_b200 import _lib
-from block_sparse_attention_cov_b200.build import build
 from block_sparse_attention_cov_b200.inputs import WORKLOADS, make_qkv
+from hooklib import hooks_lib
 from oracle import solattn_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -28,16 +28,7 @@ pytestmark = pytest.mark.gpu
 def H():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    L = ctypes.CDLL(build(hooks=True))
-    i, vp, f, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
-    L.solattn_test_set_hook.argtypes = [i, ctypes.c_ulonglong]
-    L.solattn_test_set_hook.restype = i
-    L.solattn_pooled_layout.argtypes = [i, i, i, i, vp, ctypes.POINTER(_lib.PooledStruct), ctypes.POINTER(sz)]
-    L.solattn_pool.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(_lib.PooledStruct), vp]
-    L.solattn_forward.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(_lib.PooledStruct), f, vp, vp, vp, vp, sz,
-                                  vp]
-    L.solattn_status.argtypes = [vp, vp]
-    return L
+    return hooks_lib()
 
 
 def _run(L, q, k, v, beta):
@@ -79,3 +70,25 @@ def test_expired_wait_reports_timeout_and_next_launch_succeeds(H):
     err = og - out_o
     assert np.linalg.norm(err) / np.linalg.norm(out_o) <= 1e-2 and np.abs(err).max() <= 2e-2
     assert np.abs(lse.cpu().numpy() - lse_o).max() <= 1e-3
+
+
+def test_noalloc_status_reports_an_expired_wait(H):
+    """solattn_forward_noalloc keeps its status block in the static array;
+    solattn_noalloc_status reads it back (no allocation) and reports the
+    timeout that the call's own return code cannot."""
+    wl = WORKLOADS["tiny"]
+    q, k, v = (x.cuda() for x in make_qkv(wl, seed=8))
+    B, Hh, N, d = q.shape
+    out = torch.empty_like(q)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    assert H.solattn_test_set_hook(0, 20_000_000) == 0
+    try:
+        assert H.solattn_forward_noalloc(p(q), p(k), p(v), B, Hh, N, d, 0.5, p(out), None, None, None) == 0
+        assert H.solattn_noalloc_status(None) == _lib.ERR_TIMEOUT
+    finally:
+        assert H.solattn_test_set_hook(-1, 2_000_000_000) == 0
+    assert H.solattn_forward_noalloc(p(q), p(k), p(v), B, Hh, N, d, 0.5, p(out), None, None, None) == 0
+    assert H.solattn_noalloc_status(None) == _lib.OK
+    out_o, _, _ = orc.forward(q.cpu(), k.cpu(), v.cpu(), 0.5)
+    err = out.float().cpu().numpy().astype(np.float64) - out_o
+    assert np.linalg.norm(err) / np.linalg.norm(out_o) <= 1e-2 and np.abs(err).max() <= 2e-2

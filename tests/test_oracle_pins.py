@@ -130,6 +130,20 @@ def test_beta_minus_inf_is_dense_attention():
     assert (dens == 5).all()
 
 
+@pytest.mark.parametrize("N,d,scale", [(64 * 3 + 5, 64, 1.0), (200, 128, 1.0), (130, 128, 15.0)])
+def test_dense_attention_is_library_softmax_attention(N, d, scale):
+    """dense_attention (the checker of the dense GPU path) against torch's
+    scaled_dot_product_attention and logsumexp in fp64; the large-scale case
+    has scores far from zero, so a missing max subtraction would overflow."""
+    rng = _rng(55 + N)
+    q, k, v = (scale * rng.standard_normal((N, d)) for _ in range(3))
+    out, lse = orc.dense_attention(q, k, v)
+    np.testing.assert_allclose(out, _sdpa64(q, k, v), rtol=1e-11, atol=1e-12)
+    x = (q @ k.T) / math.sqrt(d)
+    np.testing.assert_allclose(lse, torch.logsumexp(torch.as_tensor(x), dim=1).numpy(), rtol=1e-12, atol=1e-12)
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
+
+
 @pytest.mark.parametrize("beta", [-math.inf, -0.5, 0.0, 0.8, math.inf])
 def test_block_constant_inputs_make_the_correction_exact(beta):
     # With queries and keys constant inside each block, the zeroth-order Taylor
