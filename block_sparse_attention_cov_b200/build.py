@@ -17,7 +17,7 @@ LIB = os.path.join(PKG, "libsolattn.so")
 # Test-only variant (failure-detection tests): adds solattn_test_set_hook, which
 # makes one CTA skip its first K tile and shortens the bounded-wait budget.
 LIB_HOOKS = os.path.join(PKG, "libsolattn_testhooks.so")
-SOURCES = ["api.cu", "pool.cu", "forward.cu"]
+SOURCES = ["api.cu", "pool.cu", "forward.cu", "forward_pp.cu"]
 HEADERS = ["kernels.h", "ptx.cuh", "fwd_common.cuh"]
 
 NVCC_FLAGS = [

@@ -12,6 +12,10 @@
 
 namespace {
 
+#ifdef SOLATTN_TEST_HOOKS
+bool g_force_one_unit = false;  // test builds: run every forward on the one-unit kernel
+#endif
+
 using solattn::DeviceStatus;
 using solattn::PooledPtrs;
 
@@ -141,10 +145,35 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   a.d = d;
   a.st = strides;
   a.status = workspace;
-  return solattn::launch_forward(a, sms, s) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+  // the threshold rule with the block-level correction (the method) and the
+  // dense path run on the two-units-in-flight kernel; the ablation rules and
+  // the per-token correction on the one-unit kernel
+  bool pp = a.rule == SOLATTN_RULE_THRESHOLD && a.token_corr == 0;
+#ifdef SOLATTN_TEST_HOOKS
+  if (g_force_one_unit) pp = false;
+#endif
+  const cudaError_t e = pp ? solattn::launch_forward_pp(a, sms, s) : solattn::launch_forward(a, sms, s);
+  return e == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
 }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int run_pool(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+             const solattn_strides_t* strides, const solattn_pooled_t* pooled, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  solattn::Strides st;
+  if ((rc = resolve_strides(strides, B, H, N, d, &st))) return rc;
+  if ((rc = check_qkv(q, k, v))) return rc;
+  if ((rc = check_pooled(pooled))) return rc;
+  int sms = 0;
+  if ((rc = current_device_sms(&sms))) return rc;
+  const cudaError_t e =
+      solattn::launch_pool(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                           static_cast<const uint16_t*>(v), to_ptrs(pooled), B * H, H, N, d, st, sms,
+                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -205,19 +234,7 @@ int solattn_pool(const void* q, const void* k, const void* v, int B, int H, int 
 
 int solattn_pool_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                     const solattn_strides_t* strides, const solattn_pooled_t* pooled, void* stream) {
-  int rc = check_shape(B, H, N, d);
-  if (rc) return rc;
-  solattn::Strides st;
-  if ((rc = resolve_strides(strides, B, H, N, d, &st))) return rc;
-  if ((rc = check_qkv(q, k, v))) return rc;
-  if ((rc = check_pooled(pooled))) return rc;
-  int sms = 0;
-  if ((rc = current_device_sms(&sms))) return rc;
-  const cudaError_t e =
-      solattn::launch_pool(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-                           static_cast<const uint16_t*>(v), to_ptrs(pooled), B * H, H, N, d, st, sms,
-                           static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+  return run_pool(q, k, v, B, H, N, d, strides, pooled, stream);
 }
 
 int solattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
@@ -248,15 +265,26 @@ int solattn_dense(const void* q, const void* k, const void* v, int B, int H, int
 // CTA `skip_cta` never requests its first K tile (-1: none) and every bounded
 // wait gives up after `wait_budget_ns`.
 int solattn_test_set_hook(int skip_cta, unsigned long long wait_budget_ns) {
-  return solattn::set_test_hooks_fwd(skip_cta, wait_budget_ns) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+  const bool ok = solattn::set_test_hooks_fwd(skip_cta, wait_budget_ns) == cudaSuccess &&
+                  solattn::set_test_hooks_pp(skip_cta, wait_budget_ns) == cudaSuccess;
+  return ok ? SOLATTN_OK : SOLATTN_ERR_CUDA;
 }
 
 // Test builds only: every later forward copies its units' kept bitmaps to `mask`
 // ([B*H][N_b][ceil(N_b / 32)] uint32, bit j % 32 of word j / 32 = key block j
 // kept) and mu_i, sigma_i, tau_i to `stats` ([B*H][N_b][3] float; NaN where the
 // rule does not define them). NULL, NULL switches the copy off.
+// Test builds only: 1 runs every forward and dense call on the one-unit kernel
+// (forward.cu), 0 restores the normal choice.
+int solattn_test_force_one_unit(int on) {
+  g_force_one_unit = on != 0;
+  return SOLATTN_OK;
+}
+
 int solattn_test_set_route_dump(uint32_t* mask, float* stats) {
-  return solattn::set_route_dump_fwd(mask, stats) == cudaSuccess ? SOLATTN_OK : SOLATTN_ERR_CUDA;
+  const bool ok = solattn::set_route_dump_fwd(mask, stats) == cudaSuccess &&
+                  solattn::set_route_dump_pp(mask, stats) == cudaSuccess;
+  return ok ? SOLATTN_OK : SOLATTN_ERR_CUDA;
 }
 #endif
 

@@ -88,9 +88,10 @@ struct Params {
   DeviceStatus* status;
 };
 
+template <int REGION = 0>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           DeviceStatus* st, uint32_t site, uint32_t unit) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, st, site, unit);
+  const bool ok = mbar_wait<REGION>(bar, parity, abort_flag, st, site, unit);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -109,6 +110,15 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Read-only global load that does not allocate in L1: the routing warps stream
+// the head's pooled values and covariance (hundreds of KB per unit) from L2,
+// and L1 (what shared memory leaves of it) is better kept for the other warps.
+__device__ __forceinline__ float ld_stream_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
 }
 
 // Helpers of the routing warps and of the top-k / top-p cut.
@@ -183,7 +193,7 @@ __device__ bool route_unit(SM& sm, const Params& P, int s, int bh, int pair, int
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll 16
     for (int r = 0; r < D; ++r) {
-      const float c = __ldg(C + r * D + col);
+      const float c = ld_stream_f32(C + r * D + col);
       if constexpr (D == 128) {
         y0 = fmaf(sm.rq[0][r], c, y0);
         y1 = fmaf(sm.rq[1][r], c, y1);
@@ -250,7 +260,7 @@ __device__ bool route_unit(SM& sm, const Params& P, int s, int bh, int pair, int
     if (deciding) {
 #pragma unroll
       for (int jj = 0; jj < kChunk; ++jj)
-        vcur[jj] = (c * kChunk + jj < NB) ? __ldg(vb + static_cast<long long>(c * kChunk + jj) * D + vcol) : 0.f;
+        vcur[jj] = (c * kChunk + jj < NB) ? ld_stream_f32(vb + static_cast<long long>(c * kChunk + jj) * D + vcol) : 0.f;
     }
     const int j0 = c * kChunk;
     const int nk = min(kChunk, NB - j0);

@@ -45,12 +45,21 @@ struct ForwardArgs {
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, const PooledPtrs& p, int BH,
                         int H, int N, int d, const Strides& st, int num_sms, cudaStream_t stream);
 
+// Fused forward with per-unit key lists (any kept-set rule, either
+// correction): one unit in flight per CTA (forward.cu).
 cudaError_t launch_forward(const ForwardArgs& a, int num_sms, cudaStream_t stream);
+
+// Fused forward with two units in flight per CTA (forward_pp.cu): threshold
+// rule with the block-level correction (forced blocks allowed), and the dense
+// path.
+cudaError_t launch_forward_pp(const ForwardArgs& a, int num_sms, cudaStream_t stream);
 
 #ifdef SOLATTN_TEST_HOOKS
 // Test builds only: hook variables of each kernel's translation unit.
 cudaError_t set_test_hooks_fwd(int skip_cta, unsigned long long wait_budget_ns);
 cudaError_t set_route_dump_fwd(uint32_t* mask, float* stats);
+cudaError_t set_test_hooks_pp(int skip_cta, unsigned long long wait_budget_ns);
+cudaError_t set_route_dump_pp(uint32_t* mask, float* stats);
 #endif
 
 }  // namespace solattn
