@@ -539,18 +539,12 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         // ---- P with this group's reference (raised by this tile if needed),
         // one kept 64-key half at a time (P of half h over S columns
         // 32 h .. 32 h + 31; S of keys 64-127 is read before half 1's P is
-        // stored). A half the row's query block did not keep gets P = 0: those
-        // stores go first and are waited for only before P is handed to the
-        // PV (a store into a slot its QK has just written completes slowly).
-        // (columns 32-63 hold S of half 0's keys 32-63 until half 0 is read)
-        if (!kept0) tmem_st32_zero(colS);
-        if (nb == 2 && !kept1 && !kept0) tmem_st32_zero(colS + 32);
+        // stored). A half the row's query block did not keep gets P = 0 below.
         float ms = m, lt = 0.f;
         if (kept0) {
           const float2 r0 = softmax_half_tmem(colS, nv0, ms, sl2, false);
           ms = r0.x;
           lt = r0.y;
-          if (nb == 2 && !kept1) tmem_st32_zero(colS + 32);
         }
         if (kept1) {
           const float2 r1 = softmax_half_tmem(colS + 64, nv1, ms, sl2, kept0);
@@ -586,9 +580,13 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         }
         l = ((m == -INFINITY) ? 0.f : l * pow2_f32(m - mf)) + lt;
         m = mf;
-        // ---- pass the reference on (to the next tile or the end of the unit)
+        // ---- zero P for the halves not kept: issued last (a TMEM store into a
+        // slot soon after its QK completed stalls the warp), and after every
+        // read of the slot's S; then pass the reference on
+        if (!kept0) tmem_st32_zero(colS);
+        if (nb == 2 && !kept1) tmem_st32_zero(colS + 32);
         sm.xm[r] = m;
-        tmem_wait_st();  // the zero halves' stores have landed
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
