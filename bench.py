@@ -122,8 +122,8 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- traffic record
-TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "solattn_fwd_kernel.traffic.txt")
-FWD_SOURCE = os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", "forward.cu")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "solattn_fwd_pp_kernel.traffic.txt")
+FWD_SOURCE = os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", "forward_pp.cu")
 
 
 def fwd_traffic(heads):
@@ -135,7 +135,7 @@ def fwd_traffic(heads):
         rec = dict(ln.split(":", 1) for ln in open(TRAFFIC_RECORD).read().splitlines() if ":" in ln)
         rec = {k.strip(): v.strip() for k, v in rec.items()}
         digest = hashlib.sha256(open(FWD_SOURCE, "rb").read()).hexdigest()
-        if rec.get("forward_cu_sha256") != digest:
+        if rec.get("source_sha256") != digest:
             return None
         per_head = (float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])) / float(rec["heads"])
         return per_head * heads
@@ -170,12 +170,44 @@ def dense_flops(B, H, N, d):
     return 4.0 * d * N * N * B * H
 
 
+def union_flops(stats, beta, N, d, n_forced=0):
+    """Tensor-core work of the threshold rule's 128-row units (bookkeeping on
+    the pooled statistics): a unit multiplies every key block kept by either of
+    its two query blocks for all 128 rows, 4 d 128 64 FLOPs per block (QK^T and
+    PV). Its ratio to the kept-block FLOPs is what the tensor pipe does per
+    useful FLOP."""
+    qbar, kbar = stats.view("qbar").double(), stats.view("kbar").double()
+    B, H, nb, _ = qbar.shape
+    s = 1.0 / math.sqrt(d)
+    mu = s * (qbar @ stats.view("kmean").double().unsqueeze(-1)).squeeze(-1)
+    sigma = s * ((qbar @ stats.view("kcov").double()) * qbar).sum(-1).clamp_min(0.0).sqrt()
+    tau = torch.where(sigma == 0, torch.full_like(mu, math.inf), mu + beta * sigma)
+    blocks = 0.0
+    for b in range(B):
+        for h in range(H):
+            mask = (s * (qbar[b, h] @ kbar[b, h].T)) > tau[b, h].unsqueeze(-1)
+            if n_forced:
+                mask[:, :n_forced] = True
+            if nb % 2:
+                mask = torch.cat([mask, torch.zeros_like(mask[:1])])
+            blocks += float((mask[0::2] | mask[1::2]).sum().item())
+    return 4.0 * d * 128 * 64 * blocks
+
+
+def density_stats(dens, nb):
+    """Distribution of the per-row kept fraction |S_i| / N_b over every (b, h, i)."""
+    x = dens.double().flatten().cpu().numpy() / nb
+    return {"mean": float(x.mean()), "std": float(x.std()), "min": float(x.min()), "max": float(x.max()),
+            "p5": float(np.percentile(x, 5)), "p50": float(np.percentile(x, 50)), "p95": float(np.percentile(x, 95))}
+
+
 def pool_bytes(B, H, N, d):
     nb = math.ceil(N / 64)
     return 3 * B * H * N * d * 2 + (3 * nb * d + d + d * d) * B * H * 4 + 2 * nb * d * B * H * 2
 
 
 def cpu_threads():
+    """BLAS threads numpy uses (the oracle's matrix products)."""
     try:
         from threadpoolctl import threadpool_info
 
@@ -185,28 +217,111 @@ def cpu_threads():
         return 1
 
 
-def oracle_sample(q, k, v, beta, heads, blocks_per_head, seed=0):
-    """Times the oracle on a stratified sample: per head, the first and last
-    query block plus random ones. Returns (seconds, kept FLOPs of the sample,
-    description)."""
+def cpu_info():
+    """Cores this process may run on, the CPU model and the BLAS threads."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cores": len(os.sched_getaffinity(0)), "cpu_model": model, "blas_threads": cpu_threads()}
+
+
+SAMPLE_BLOCKS = 32  # per head: the first and last query block and 30 seeded random ones
+
+
+def sample_rows(nb, head, seed=0):
+    """The stratified sample of query blocks of one head."""
+    rng = np.random.default_rng(seed * 100003 + head)
+    inner = np.arange(1, nb - 1)  # the random ones are drawn between the first and the last
+    extra = rng.choice(inner, min(len(inner), SAMPLE_BLOCKS - 2), replace=False).tolist() if len(inner) else []
+    return sorted({0, nb - 1, *extra})
+
+
+def row_kept_flops(mask, N, d):
+    """Kept-block FLOPs of every query block i: 4 d n_i sum_{j in S_i} n_j."""
+    from oracle import solattn_oracle as orc
+
+    n = orc.block_counts(N).astype(np.float64)
+    return 4.0 * d * n * (mask.astype(np.float64) @ n)
+
+
+def oracle_head_sample(q, k, v, beta, head_pos, head_id, seed=0):
+    """The oracle (fp32 working precision, multithreaded BLAS) on the stratified
+    sample of one head. Returns (seconds, kept FLOPs of the sample)."""
     from oracle import solattn_oracle as orc
 
     N, d = q.shape[2], q.shape[3]
     nb = math.ceil(N / 64)
-    rng = np.random.default_rng(seed)
-    t_total, flops = 0.0, 0.0
-    for h in heads:
-        rows = sorted({0, nb - 1, *rng.choice(nb, max(0, blocks_per_head - 2), replace=False).tolist()})
-        qq, kk, vv = (x[0, h].double().numpy() for x in (q, k, v))
+    rows = sample_rows(nb, head_id, seed)
+    qq, kk, vv = (x[0, head_pos].float().numpy() for x in (q, k, v))
+    t0 = time.perf_counter()
+    orc.attend(qq, kk, vv, beta, rows=rows, dtype=np.float32)
+    secs = time.perf_counter() - t0
+    r = orc.route(qq, kk, beta, dtype=np.float32)
+    return secs, float(row_kept_flops(r["mask"], N, d)[rows].sum())
+
+
+def routing_oracle(q, k, beta, dens_gpu):
+    """The routing oracle (fp64) over every query block of every head: time,
+    near ties (|s_hat - tau| <= 1e-4), query blocks whose GPU kept count
+    differs from the oracle's by more than their near ties, and the kept FLOPs
+    of every row (for the extrapolation of the CPU time)."""
+    from oracle import solattn_oracle as orc
+
+    B, H, N, d = q.shape
+    secs, ties, bad, flops = 0.0, 0, 0, []
+    for h in range(H):
+        qq, kk = q[0, h].double().numpy(), k[0, h].double().numpy()
         t0 = time.perf_counter()
-        _, _, dens = orc.attend(qq, kk, vv, beta, rows=rows)
-        t_total += time.perf_counter() - t0
         r = orc.route(qq, kk, beta)
-        n = orc.block_counts(N).astype(np.float64)
-        for i in rows:
-            flops += 4.0 * d * n[i] * float(n[r["mask"][i]].sum())
-    desc = f"oracle fp64 on {len(heads)} head(s) x {blocks_per_head} query blocks (first, last, random)"
-    return t_total, flops, desc
+        secs += time.perf_counter() - t0
+        near = (np.abs(r["shat"] - r["tau"][:, None]) <= 1e-4).sum(1)
+        ties += int(near.sum())
+        bad += int((np.abs(dens_gpu[0, h].astype(np.int64) - r["density"]) > near).sum())
+        flops.append(row_kept_flops(r["mask"], N, d))
+    return secs, ties, bad, np.stack(flops)
+
+
+def cpu_baseline_leg(q, k, v, beta, dens_gpu, seed=0):
+    """CPU baseline as the oracle stands: fp32 multithreaded BLAS on the
+    stratified sample of every head (first, last, 30 random query blocks),
+    with the full forward's CPU time extrapolated from it by kept FLOPs; the
+    routing oracle over every block (also the near-tie and kept-count parity
+    of the GPU run); the tiny and mid workloads timed in full."""
+    from oracle import solattn_oracle as orc
+
+    B, H, N, d = q.shape
+    nb = math.ceil(N / 64)
+    r_secs, ties, bad, row_flops = routing_oracle(q, k, beta, dens_gpu)
+    s_secs, s_flops = 0.0, 0.0
+    for h in range(H):
+        t, f = oracle_head_sample(q, k, v, beta, h, h, seed)
+        s_secs += t
+        s_flops += f
+    total_flops = float(row_flops.sum())
+    full = {}
+    for name, wl_beta in (("tiny", 1.0), ("mid", 1.0)):
+        wl = WORKLOADS[name]
+        qt, kt, vt = make_qkv(wl, seed=0)
+        t0 = time.perf_counter()
+        for h in range(wl.H):
+            orc.attend(*(x[0, h].float().numpy() for x in (qt, kt, vt)), wl_beta, dtype=np.float32)
+        full[name] = {"seconds": round(time.perf_counter() - t0, 3), "beta": wl_beta, "heads": wl.H, "N": wl.N}
+    info = cpu_info()
+    return {
+        "value": s_flops / s_secs / 1e12, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+        "sample": f"oracle fp32, {H} heads x {SAMPLE_BLOCKS} query blocks (first, last, 30 seeded random); "
+                  f"{s_secs:.1f} s of CPU time",
+        "cpu_model": info["cpu_model"], "blas_threads": info["blas_threads"],
+        "sample_seconds": s_secs, "sample_kept_tflop": s_flops / 1e12,
+        "full_forward_seconds_extrapolated": s_secs * total_flops / s_flops,
+        "routing_oracle_seconds_all_blocks": r_secs,
+        "full_runs": full,
+    }, {"near_ties": ties, "density_mismatch_rows": bad, "rows": int(H * nb)}
 
 
 def max_over_ranks(values, world, device):
@@ -226,26 +341,37 @@ def job_value(flops_per_rank, ms, world):
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
+    """The oracle as it stands (fp32 working precision, multithreaded BLAS) on
+    the host cores. Step s times the stratified sample of head s % H (first,
+    last and 30 seeded random query blocks): the same per-head samples the
+    cpu_baseline leg of the GPU arm times for every head."""
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
     beta = args.beta if args.beta is not None else load_beta(args.workload, args.density)[0]
-    q, k, v = make_qkv(wl, 0, heads=[(0, 0)])
+    heads = sorted({s_ % wl.H for s_ in range(args.warmup + args.steps)})
+    q, k, v = make_qkv(wl, 0, heads=[(0, h) for h in heads])
+    pos = {h: i for i, h in enumerate(heads)}
     times, flops = [], 0.0
     for step in range(args.warmup + args.steps):
-        t, f, desc = oracle_sample(q, k, v, beta, [0], 4, seed=step)
+        h = step % wl.H
+        t, f = oracle_head_sample(q, k, v, beta, pos[h], h)
         if step >= args.warmup:
             times.append(t)
             flops += f
     secs = sum(times)
     val = flops / secs / 1e12
+    info = cpu_info()
+    desc = (f"oracle fp32 per step: {SAMPLE_BLOCKS} query blocks (first, last, 30 seeded random) of head "
+            f"step % {wl.H}; {secs:.1f} s of CPU time over {args.steps} steps")
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": args.workload, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "beta": beta,
                    "sample": desc},
-        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": desc,
+                         "cpu_model": info["cpu_model"], "blas_threads": info["blas_threads"]},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -392,11 +518,10 @@ def run_ours(args, rank, world, local_rank):
         peak_tc, peak_kind = peaks["bf16_tflops"], " (bf16 burst)"
     pbytes = pool_bytes(B, H, N, d)
     pool_gbs = pbytes / (pool_ms * 1e-3) / 1e9
-    cpu = None
-    if not args.skip_cpu and world == 1:
-        secs, fl, desc = oracle_sample(q_h, k_h, v_h, beta, [0, H // 2], args.cpu_blocks)
-        cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": desc + f"; {secs:.1f} s of CPU time"}
+    cpu, parity = None, None
+    if not args.skip_cpu and world == 1 and args.rule == "threshold" and not args.n_forced:
+        cpu, parity = cpu_baseline_leg(q_h, k_h, v_h, beta, dens.cpu().numpy())
+    uflops = union_flops(stats, beta, N, d, args.n_forced) if args.rule == "threshold" else None
     line = {
         "metric": METRIC,
         "value": job_value(kflops, ms_step, world),
@@ -430,6 +555,11 @@ def run_ours(args, rank, world, local_rank):
         "dense_ms": dense_ms,
         "speedup_vs_dense": (dense_ms / fwd_ms) if dense_ms else None,
         "kept_tflop_per_step": kflops / 1e12,
+        "union_tflop_per_step": None if uflops is None else uflops / 1e12,
+        "pair_efficiency": None if uflops is None else kflops / uflops,
+        "density": density_stats(dens, nb),
+        "near_ties": None if parity is None else parity["near_ties"],
+        "density_mismatch_rows": None if parity is None else parity["density_mismatch_rows"],
         "roofline": {
             "bound": "tensor",
             "achieved": fwd_tflops,
@@ -437,7 +567,7 @@ def run_ours(args, rank, world, local_rank):
             "unit": "TFLOP/s",
             "frac": fwd_tflops / peak_tc,
             "traffic": fwd_traffic(B * H),
-            "kernel": "solattn_fwd_kernel (fused forward)",
+            "kernel": "solattn_fwd_pp_kernel (fused forward)",
             "peak_source": peaks["source"] + peak_kind,
         },
         "pool_roofline": {
@@ -454,6 +584,82 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- suite
+def run_suite(args):
+    """One JSON line per configuration of the length sweep (16K-128K tokens x
+    5/10/15/30 % density, 24 heads), the HunyuanVideo-like attention (10 / 15
+    %) and the kept-set rules at the Wan-like 15 % (threshold, top-k, top-p):
+    forward ms, kept-block TFLOP/s and its fraction of the bf16 burst peak, the
+    dense path's ms and the speed-up, the per-row density distribution and the
+    clocks of each timed loop. Inputs resident on the GPU; 3 warm-up and 5
+    timed forwards per configuration."""
+    import block_sparse_attention_cov_b200 as sa
+    from block_sparse_attention_cov_b200 import _lib
+
+    _lib.lib()
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+
+    def timed(fn, reps, warm=2):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(cvd.split(",")[0] if cvd else "0")
+        clocks.start()
+        time.sleep(0.2)
+        w0 = time.monotonic()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark(w0, time.monotonic())
+        return e0.elapsed_time(e1) / reps, clocks.stop()
+
+    plan = [(name, None) for name in ("sweep_16k", "sweep_32k", "sweep_64k", "sweep_128k", "hunyuan_119k")]
+    plan.append(("wan_75k", "rules"))
+    for name, mode in plan:
+        wl = WORKLOADS[name]
+        q, k, v = (x.to(dev) for x in make_qkv(wl, seed=0))
+        B, H, N, d = q.shape
+        nb = math.ceil(N / 64)
+        ws = sa.workspace(dev)
+        stats = sa.pool(q, k, v)
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dens = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+        dense_ms, _ = timed(lambda: sa.dense(q, k, v, out=out, lse=lse, ws=ws), 2, 1)
+        beta15 = load_beta(name, 0.15)[0]
+        if mode == "rules":
+            runs = [("threshold", {"rule": "threshold"}, beta15),
+                    ("topk", {"rule": "topk", "topk": args.topk}, 0.0),
+                    ("topp", {"rule": "topp", "topp": args.topp}, 0.0)]
+        else:
+            targets = json.load(open(os.path.join(ROOT, "tests", "golden", "calibrated_beta.json")))[name]["targets"]
+            runs = [(f"{float(t):.0%}", {"rule": "threshold"}, targets[t]["beta"]) for t in sorted(targets)]
+        for label, kw, beta in runs:
+            fwd = lambda: sa.forward(q, k, v, stats, beta, out=out, lse=lse, density=dens, ws=ws, **kw)
+            ms, clk = timed(fwd, 5, 3)
+            if sa.status(ws) != 0:
+                raise RuntimeError(f"device status {sa.status(ws)} in {name} {label}")
+            kfl = kept_flops(stats, dens, beta, N, d, kw["rule"])
+            tf = kfl / (ms * 1e-3) / 1e12
+            line = {"suite": name, "config": label, "rule": kw["rule"], "beta": beta,
+                    **({"topk": kw["topk"]} if "topk" in kw else {}), **({"topp": kw["topp"]} if "topp" in kw else {}),
+                    "B": B, "H": H, "N": N, "d": d, "fwd_ms": ms, "kept_tflop": kfl / 1e12, "kept_tflops": tf,
+                    "frac_bf16_burst": tf / peaks["bf16_tflops"], "dense_ms": dense_ms,
+                    "speedup_vs_dense": dense_ms / ms, "density": density_stats(dens, nb), "clocks": clk}
+            if kw["rule"] == "threshold":
+                uf = union_flops(stats, beta, N, d)
+                line["pair_efficiency"] = kfl / uf
+            print(json.dumps(line), flush=True)
+        del q, k, v, stats, out, lse, dens
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -465,7 +671,6 @@ def main():
     ap.add_argument("--density", type=float, default=None,
                     help="use the calibrated beta of this mean kept-block density (e.g. 0.05 on the sweeps)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
-    ap.add_argument("--cpu-blocks", type=int, default=600)
     ap.add_argument("--rule", choices=["threshold", "topk", "topp"], default="threshold",
                     help="kept-set rule (the method is 'threshold'; top-k / top-p are the ablation rules)")
     ap.add_argument("--topk", type=int, default=177, help="top-k rule: blocks per query block (15 %% of 1182)")
@@ -477,6 +682,8 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-dense", action="store_true")
+    ap.add_argument("--suite", action="store_true",
+                    help="one JSON line per configuration of the sweep, the Hunyuan-like workload and the rules")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -491,7 +698,9 @@ def main():
             torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     try:
-        if args.impl == "reference":
+        if args.suite:
+            run_suite(args)
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local_rank)

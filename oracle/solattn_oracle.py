@@ -102,10 +102,10 @@ def block_counts(N: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Step 2: block means
 # --------------------------------------------------------------------------
-def pool(x: np.ndarray) -> np.ndarray:
+def pool(x: np.ndarray, dtype=np.float64) -> np.ndarray:
     """Block means over valid tokens: x [N, d] -> x_bar [N_b, d]."""
-    x = np.asarray(x, dtype=np.float64)
-    out = np.empty((len(block_bounds(x.shape[0])), x.shape[1]), dtype=np.float64)
+    x = np.asarray(x, dtype=dtype)
+    out = np.empty((len(block_bounds(x.shape[0])), x.shape[1]), dtype=dtype)
     for b, (start, stop) in enumerate(block_bounds(x.shape[0])):
         out[b] = x[start:stop].sum(axis=0) / (stop - start)
     return out
@@ -114,10 +114,10 @@ def pool(x: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Step 3: key statistics
 # --------------------------------------------------------------------------
-def key_stats(kbar: np.ndarray):
+def key_stats(kbar: np.ndarray, dtype=np.float64):
     """Mean k_mean [d] and covariance C [d, d] of the pooled keys, population
     normalisation (divide by N_b), two-pass."""
-    kbar = np.asarray(kbar, dtype=np.float64)
+    kbar = np.asarray(kbar, dtype=dtype)
     nb = kbar.shape[0]
     kmean = kbar.sum(axis=0) / nb
     dev = kbar - kmean
@@ -128,9 +128,9 @@ def key_stats(kbar: np.ndarray):
 # --------------------------------------------------------------------------
 # Step 4: per-row mean and standard deviation of the proxy scores
 # --------------------------------------------------------------------------
-def row_stats(qbar: np.ndarray, kmean: np.ndarray, kcov: np.ndarray):
+def row_stats(qbar: np.ndarray, kmean: np.ndarray, kcov: np.ndarray, dtype=np.float64):
     """mu_i = s q_bar_i . k_mean,  sigma_i = s sqrt(q_bar_i^T C q_bar_i)."""
-    qbar = np.asarray(qbar, dtype=np.float64)
+    qbar = np.asarray(qbar, dtype=dtype)
     s = 1.0 / math.sqrt(qbar.shape[1])
     mu = s * (qbar @ kmean)
     quad = np.einsum("id,de,ie->i", qbar, kcov, qbar)
@@ -156,24 +156,24 @@ def thresholds(mu: np.ndarray, sigma: np.ndarray, beta: float) -> np.ndarray:
     return np.where(sigma == 0.0, math.inf, mu + beta * sigma)
 
 
-def proxy_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+def proxy_scores(qbar: np.ndarray, kbar: np.ndarray, dtype=np.float64) -> np.ndarray:
     """s_hat_ij = q_bar_i . k_bar_j / sqrt(d) (the oracle may form the whole row;
     the method itself never writes it out)."""
     s = 1.0 / math.sqrt(qbar.shape[1])
-    return s * (np.asarray(qbar, np.float64) @ np.asarray(kbar, np.float64).T)
+    return s * (np.asarray(qbar, dtype) @ np.asarray(kbar, dtype).T)
 
 
-def route(q: np.ndarray, k: np.ndarray, beta: float) -> dict:
+def route(q: np.ndarray, k: np.ndarray, beta: float, dtype=np.float64) -> dict:
     """Routing only (steps 1-5) for one head: q, k [N, d].
 
     Returns s_hat [N_b, N_b], tau [N_b], mu, sigma, mask [N_b, N_b] (bool,
     True = kept), density [N_b] (= |S_i|), plus the pooled statistics.
     """
-    qbar, kbar = pool(q), pool(k)
-    kmean, kcov = key_stats(kbar)
-    mu, sigma = row_stats(qbar, kmean, kcov)
+    qbar, kbar = pool(q, dtype), pool(k, dtype)
+    kmean, kcov = key_stats(kbar, dtype)
+    mu, sigma = row_stats(qbar, kmean, kcov, dtype)
     tau = thresholds(mu, sigma, beta)
-    shat = proxy_scores(qbar, kbar)
+    shat = proxy_scores(qbar, kbar, dtype)
     mask = shat > tau[:, None]
     return {
         "qbar": qbar,
@@ -258,7 +258,7 @@ def route_rule(q: np.ndarray, k: np.ndarray, rule: str, param: float, n_forced: 
 # --------------------------------------------------------------------------
 # Step 6: attention with exact kept blocks and zeroth-order correction
 # --------------------------------------------------------------------------
-def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None, correction: str = "block"):
+def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None, correction: str = "block", dtype=np.float64):
     """Sol-Attn forward for one head, offline threshold form.
 
     q, k, v: [N, d]. mask: optional [N_b, N_b] bool to use instead of the
@@ -269,26 +269,27 @@ def attend(q, k, v, beta: float = -math.inf, mask=None, rows=None, correction: s
     calcola": every token of the skipped block is taken to carry the block's
     mean key, so row t scores it s q_t . kbar_j; the value is still vbar_j).
     Returns out [N, d], lse [N] (natural log of the softmax denominator of the
-    scaled scores), density [N_b] (= |S_i|).
+    scaled scores), density [N_b] (= |S_i|). dtype: the working precision
+    (fp64 for every parity check; fp32 only to time the CPU baseline).
     """
     if correction not in ("block", "token"):
         raise ValueError(correction)
-    q = np.asarray(q, np.float64)
-    k = np.asarray(k, np.float64)
-    v = np.asarray(v, np.float64)
+    q = np.asarray(q, dtype)
+    k = np.asarray(k, dtype)
+    v = np.asarray(v, dtype)
     N, d = q.shape
     s = 1.0 / math.sqrt(d)
     bounds = block_bounds(N)
-    n = block_counts(N).astype(np.float64)
-    r = route(q, k, beta)
+    n = block_counts(N).astype(dtype)
+    r = route(q, k, beta, dtype)
     shat = r["shat"]
-    vbar = pool(v)
+    vbar = pool(v, dtype)
     kbar = r["kbar"]
     if mask is None:
         mask = r["mask"]
     mask = np.asarray(mask, dtype=bool)
-    out = np.full((N, d), np.nan)
-    lse = np.full((N,), np.nan)
+    out = np.full((N, d), np.nan, dtype=dtype)
+    lse = np.full((N,), np.nan, dtype=dtype)
     rows = range(len(bounds)) if rows is None else rows
     for i in rows:
         a, b = bounds[i]

@@ -33,3 +33,30 @@ def test_density_picks_that_target(name):
 def test_unknown_density_is_an_error():
     with pytest.raises(KeyError):
         bench.load_beta("wan_75k", 0.42)
+
+
+def test_stratified_sample_rows():
+    """First, last and 30 seeded random query blocks per head; the same rows
+    for the same head in both CPU arms (cpu_baseline leg and --impl reference)."""
+    rows = bench.sample_rows(1182, 7)
+    assert rows[0] == 0 and rows[-1] == 1181 and len(rows) == bench.SAMPLE_BLOCKS == 32
+    assert rows == bench.sample_rows(1182, 7) and rows != bench.sample_rows(1182, 8)
+    assert bench.sample_rows(3, 0) == [0, 1, 2] and bench.sample_rows(1, 0) == [0]
+
+
+def test_row_kept_flops_counts_partial_blocks():
+    import numpy as np
+
+    # N = 150: blocks of 64, 64, 22 tokens; d = 4
+    mask = np.array([[True, False, True], [False, False, False], [True, True, True]])
+    f = bench.row_kept_flops(mask, 150, 4)
+    assert f.tolist() == [4 * 4 * 64 * (64 + 22), 0.0, 4 * 4 * 22 * 150]
+
+
+def test_density_stats():
+    import torch
+
+    dens = torch.tensor([[[1, 2, 3, 4]]], dtype=torch.int32)
+    st = bench.density_stats(dens, 8)
+    assert st["mean"] == pytest.approx(2.5 / 8) and st["min"] == 1 / 8 and st["max"] == 4 / 8
+    assert st["p50"] == pytest.approx(2.5 / 8)

@@ -331,7 +331,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert brute_pin_fails(math.inf)
     monkeypatch.undo()
     # 2. proxy score without the 1/sqrt(d) scale
-    monkeypatch.setattr(orc, "proxy_scores", lambda a, b: np.asarray(a) @ np.asarray(b).T)
+    monkeypatch.setattr(orc, "proxy_scores", lambda a, b, dtype=np.float64: np.asarray(a) @ np.asarray(b).T)
     assert brute_pin_fails(0.0)
     monkeypatch.undo()
     # 3. threshold with the sign of beta flipped
@@ -341,7 +341,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # 4. sample (ddof=1) covariance: the explicit-row invariant catches it
     real_stats = orc.key_stats
 
-    def ddof1(kbar):
+    def ddof1(kbar, dtype=np.float64):
         km, kc = real_stats(kbar)
         return km, kc * kbar.shape[0] / (kbar.shape[0] - 1)
 
