@@ -15,6 +15,10 @@ Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
 GPU (heads are independent; no collective on the data path); timing is the max
 over ranks.
 
+e2e = the same step through solattn_forward_host: q, k, v in pinned host
+memory, out, lse and density back to pinned host memory, the copies inside the
+timed region (overlapped with the computation of other head chunks).
+
 --impl reference runs the CPU oracle (the only other implementation of this
 method available here) on the host cores, on a bounded sample of the same
 workload per step.
@@ -468,28 +472,25 @@ def run_ours(args, rank, world, local_rank):
         step()  # restore the Sol-Attn outputs
         torch.cuda.synchronize()
 
-    # end to end: pinned host inputs -> device -> pool + forward -> host outputs
+    # end to end through the C ABI's host-buffer entry point (solattn_forward_host):
+    # pinned host inputs in, pinned host outputs back, copies overlapped with
+    # the pool + forward of other head chunks
     e2e = None
-    if not args.skip_e2e:
+    if not args.skip_e2e and args.rule == "threshold" and args.n_forced == 0 and args.correction == "block":
         qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         dens_h = torch.empty(dens.shape, dtype=dens.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        scratch = sa.host_scratch(B, H, N, d, device=dev)
 
         def e2e_step():
-            qd.copy_(qp, non_blocking=True)
-            kd.copy_(kp, non_blocking=True)
-            vd.copy_(vp, non_blocking=True)
-            sa.pool(qd, kd, vd, stats)
-            sa.forward(qd, kd, vd, stats, beta, out=out, lse=lse, density=dens, ws=ws, **rule_kw)
-            out_h.copy_(out, non_blocking=True)
-            lse_h.copy_(lse, non_blocking=True)
-            dens_h.copy_(dens, non_blocking=True)
+            sa.forward_host(qp, kp, vp, beta, out_h, lse_h, dens_h, scratch=scratch)
 
         e2e_step()
         torch.cuda.synchronize()
-        reps = max(1, min(args.steps, 3))
+        if sa.status(scratch) != 0:
+            raise RuntimeError(f"device status {sa.status(scratch)} in the end-to-end path")
+        reps = max(1, min(args.steps, 5))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             torch.distributed.barrier()
@@ -499,11 +500,18 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
+        if sa.status(scratch) != 0:
+            raise RuntimeError(f"device status {sa.status(scratch)} in the end-to-end path")
+        if not torch.equal(dens_h, dens.cpu()):
+            raise RuntimeError("end-to-end density differs from the device path")
         (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp))
         d2h = sum(x.numel() * x.element_size() for x in (out_h, lse_h, dens_h))
         e2e = {"value": job_value(kflops, e2e_ms, world), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "path": "solattn_forward_host: pinned host buffers, head chunks copied in / attended / "
+                       "copied back on three streams"}
+        del scratch
 
     if rank != 0:
         return
@@ -591,8 +599,10 @@ def run_suite(args):
     %) and the kept-set rules at the Wan-like 15 % (threshold, top-k, top-p):
     forward ms, kept-block TFLOP/s and its fraction of the bf16 burst peak, the
     dense path's ms and the speed-up, the per-row density distribution and the
-    clocks of each timed loop. Inputs resident on the GPU; 3 warm-up and 5
-    timed forwards per configuration."""
+    clocks of each timed loop, and for the threshold rule the near ties and the
+    rows whose kept count differs from the fp64 routing oracle. Inputs resident
+    on the GPU; warm-up calls, then a timed loop of at least 5 calls and about
+    0.8 s (so that the clock sampler sees it several times)."""
     import block_sparse_attention_cov_b200 as sa
     from block_sparse_attention_cov_b200 import _lib
 
@@ -602,10 +612,16 @@ def run_suite(args):
     stream = torch.cuda.current_stream()
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
 
-    def timed(fn, reps, warm=2):
+    def timed(fn, reps, warm=2, window_ms=800.0):
         for _ in range(warm):
             fn()
         torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        reps = max(reps, math.ceil(window_ms / max(e0.elapsed_time(e1), 1e-3)))
         clocks = ClockSampler(cvd.split(",")[0] if cvd else "0")
         clocks.start()
         time.sleep(0.2)
@@ -623,7 +639,8 @@ def run_suite(args):
     plan.append(("wan_75k", "rules"))
     for name, mode in plan:
         wl = WORKLOADS[name]
-        q, k, v = (x.to(dev) for x in make_qkv(wl, seed=0))
+        q_h, k_h, v_h = make_qkv(wl, seed=0)
+        q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
         B, H, N, d = q.shape
         nb = math.ceil(N / 64)
         ws = sa.workspace(dev)
@@ -655,8 +672,10 @@ def run_suite(args):
             if kw["rule"] == "threshold":
                 uf = union_flops(stats, beta, N, d)
                 line["pair_efficiency"] = kfl / uf
+                _, ties, bad, _ = routing_oracle(q_h, k_h, beta, dens.cpu().numpy())
+                line["near_ties"], line["density_mismatch_rows"] = ties, bad
             print(json.dumps(line), flush=True)
-        del q, k, v, stats, out, lse, dens
+        del q, k, v, q_h, k_h, v_h, stats, out, lse, dens
         torch.cuda.empty_cache()
 
 

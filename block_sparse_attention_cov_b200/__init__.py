@@ -8,6 +8,7 @@ CPU path. The names mirror the C calls:
     stats = pool(q, k, v)                          # solattn_pool
     out, lse, density = forward(q, k, v, stats, beta)   # solattn_forward
     out, lse = dense(q, k, v)                      # solattn_dense
+    forward_host(q_h, k_h, v_h, beta, out_h, ...)  # solattn_forward_host (host tensors)
 
 q, k, v: CUDA bf16 tensors [B, H, N, d], contiguous, d in {64, 128}.
 """
@@ -21,7 +22,8 @@ import torch
 
 from . import _lib
 
-__all__ = ["SolAttnError", "PooledStats", "pool", "forward", "dense", "status", "workspace", "pooled_bytes"]
+__all__ = ["SolAttnError", "PooledStats", "pool", "forward", "dense", "status", "workspace", "pooled_bytes",
+           "host_scratch", "forward_host"]
 
 
 class SolAttnError(RuntimeError):
@@ -188,6 +190,43 @@ def dense(q, k, v, out=None, lse=None, ws=None, want_lse: bool = True):
                                   ws.numel(), _stream())
     _check(rc, "solattn_dense")
     return out, lse
+
+
+def host_scratch(B: int, H: int, N: int, d: int, chunk_heads: int = 0, device=None) -> torch.Tensor:
+    """Device scratch for forward_host (solattn_host_scratch_bytes bytes)."""
+    n = ctypes.c_size_t(0)
+    _check(_lib.lib().solattn_host_scratch_bytes(B, H, N, d, int(chunk_heads), ctypes.byref(n)),
+           "solattn_host_scratch_bytes")
+    return torch.empty(n.value, dtype=torch.uint8, device=device or "cuda")
+
+
+def forward_host(q, k, v, beta: float, out, lse=None, density=None, scratch=None, chunk_heads: int = 0):
+    """solattn_forward_host: the threshold-rule forward on HOST tensors (CPU,
+    contiguous bf16 [B, H, N, d]; page-locked for the copies to overlap the
+    computation). out (bf16, q's shape), lse (float32 [B, H, N]) and density
+    (int32 [B, H, N_b]) are host tensors written once the current stream has
+    completed; the call only enqueues. scratch: a device tensor from
+    host_scratch() (allocated here when None). Returns the scratch, whose first
+    bytes hold the device status (status(scratch))."""
+    for t in (q, k, v, out):
+        if t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError("q, k, v, out must be contiguous host bf16 [B, H, N, d] tensors")
+    if not (q.shape == k.shape == v.shape == out.shape):
+        raise ValueError("q, k, v and out must have the same shape")
+    B, H, N, d = _shape(q)
+    nb = (N + _lib.BLOCK - 1) // _lib.BLOCK
+    if lse is not None and (lse.is_cuda or lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
+                            or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous host float32 [B, H, N] tensor")
+    if density is not None and (density.is_cuda or density.dtype != torch.int32 or tuple(density.shape) != (B, H, nb)
+                                or not density.is_contiguous()):
+        raise ValueError("density must be a contiguous host int32 [B, H, N_b] tensor")
+    scratch = host_scratch(B, H, N, d, chunk_heads) if scratch is None else scratch
+    rc = _lib.lib().solattn_forward_host(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, ctypes.c_float(beta), _ptr(out),
+                                         _ptr(lse), _ptr(density), int(chunk_heads), _ptr(scratch), scratch.numel(),
+                                         _stream())
+    _check(rc, "solattn_forward_host")
+    return scratch
 
 
 def status(ws: torch.Tensor) -> int:

@@ -19,6 +19,8 @@ EXPORTS = (
     "solattn_forward_ex",
     "solattn_pool_ex",
     "solattn_noalloc_status",
+    "solattn_host_scratch_bytes",
+    "solattn_forward_host",
 )
 
 OK = 0
@@ -85,6 +87,10 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.solattn_pool_ex.argtypes = [vp, vp, vp, i, i, i, i, ctypes.POINTER(StridesStruct), ctypes.POINTER(PooledStruct),
                                   vp]
     L.solattn_pool_ex.restype = i
+    L.solattn_host_scratch_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(sz)]
+    L.solattn_host_scratch_bytes.restype = i
+    L.solattn_forward_host.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, i, vp, sz, vp]
+    L.solattn_forward_host.restype = i
     L.solattn_version.argtypes = []
     L.solattn_version.restype = i
     return L

@@ -98,9 +98,11 @@ PooledPtrs to_ptrs(const solattn_pooled_t* p) {
                     static_cast<uint16_t*>(p->vbar16)};
 }
 
+// reset_status: false leaves the status word as it is (only the scheduler
+// counter restarts), so that a sequence of calls keeps the first error.
 int run_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                 const solattn_pooled_t* pooled, const solattn_options_t& opt, bool route, void* out, float* lse,
-                int32_t* density, void* workspace, size_t workspace_bytes, void* stream) {
+                int32_t* density, void* workspace, size_t workspace_bytes, void* stream, bool reset_status = true) {
   const float beta = opt.beta;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
@@ -122,8 +124,9 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   int sms = 0;
   if ((rc = current_device_sms(&sms))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // scheduler counter and status word start at zero for every call
-  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), s) != cudaSuccess) return SOLATTN_ERR_CUDA;
+  // the scheduler counter (and, normally, the status word) start at zero
+  if (cudaMemsetAsync(workspace, 0, reset_status ? sizeof(DeviceStatus) : sizeof(unsigned int), s) != cudaSuccess)
+    return SOLATTN_ERR_CUDA;
   solattn::ForwardArgs a{};
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(k);
@@ -146,8 +149,8 @@ int run_forward(const void* q, const void* k, const void* v, int B, int H, int N
   a.st = strides;
   a.status = workspace;
   // the threshold rule with the block-level correction (the method) and the
-  // dense path run on the two-units-in-flight kernel; the ablation rules and
-  // the per-token correction on the one-unit kernel
+  // dense path run on the two-group kernel (forward_pp.cu); the ablation rules
+  // and the per-token correction on the one-unit kernel (forward.cu)
   bool pp = a.rule == SOLATTN_RULE_THRESHOLD && a.token_corr == 0;
 #ifdef SOLATTN_TEST_HOOKS
   if (g_force_one_unit) pp = false;
@@ -358,6 +361,174 @@ int solattn_noalloc_status(void* stream) {
   // symbol allocates nothing
   if (cudaMemcpyFromSymbol(&h, g_noalloc_scratch, sizeof(h)) != cudaSuccess) return SOLATTN_ERR_CUDA;
   return h.error == 0 ? SOLATTN_OK : static_cast<int>(h.error);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// End-to-end forward on host buffers: the B*H (b, h) pairs go through the
+// device in chunks, double-buffered in the caller's scratch. Three streams:
+// copies to the device, the caller's stream (pool + forward), copies back;
+// events order chunk i's copy in after chunk i - 2 has left the same buffer.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct HostChunkLayout {
+  size_t q, k, v, out, lse, dens, pooled;  // offsets inside one buffer
+  size_t buffer;                           // bytes of one buffer
+  size_t pooled_bytes;
+};
+
+int default_chunk_heads(int BH) {
+  // about 16 chunks: the copy-in of the first and the copy-back of the last
+  // chunk are the only transfers not hidden behind other work
+  const int c = (BH + 15) / 16;
+  return c < 1 ? 1 : c;
+}
+
+int host_chunk_layout(int N, int d, int C, HostChunkLayout* L) {
+  size_t pooled_bytes = 0;
+  int rc = solattn_pooled_layout(1, C, N, d, nullptr, nullptr, &pooled_bytes);
+  if (rc) return rc;
+  const size_t nb = (static_cast<size_t>(N) + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
+  const size_t tensor = static_cast<size_t>(C) * N * d * 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += round256(bytes);
+    return at;
+  };
+  L->q = take(tensor);
+  L->k = take(tensor);
+  L->v = take(tensor);
+  L->out = take(tensor);
+  L->lse = take(static_cast<size_t>(C) * N * sizeof(float));
+  L->dens = take(static_cast<size_t>(C) * nb * sizeof(int32_t));
+  L->pooled = take(pooled_bytes);
+  L->buffer = off;
+  L->pooled_bytes = pooled_bytes;
+  return SOLATTN_OK;
+}
+
+// Streams and events of one solattn_forward_host call; released at the end of
+// the call (the runtime defers the release until their work has completed).
+struct HostPipeline {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t ev[3][4] = {};  // [copied in, computed, copied back][chunk % 4]
+  bool ok = true;
+  HostPipeline() {
+    ok = cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&start, cudaEventDisableTiming) == cudaSuccess;
+    for (auto& row : ev)
+      for (auto& e : row) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+  }
+  ~HostPipeline() {
+    for (auto& row : ev)
+      for (auto& e : row)
+        if (e) cudaEventDestroy(e);
+    if (start) cudaEventDestroy(start);
+    if (up) cudaStreamDestroy(up);
+    if (down) cudaStreamDestroy(down);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+int solattn_host_scratch_bytes(int B, int H, int N, int d, int chunk_heads, size_t* bytes) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (!bytes || chunk_heads < 0) return SOLATTN_ERR_ARG;
+  const int BH = B * H;
+  const int C = chunk_heads == 0 ? default_chunk_heads(BH) : (chunk_heads < BH ? chunk_heads : BH);
+  HostChunkLayout L;
+  if ((rc = host_chunk_layout(N, d, C, &L))) return rc;
+  *bytes = SOLATTN_WORKSPACE_BYTES + 2 * L.buffer;
+  return SOLATTN_OK;
+}
+
+int solattn_forward_host(const void* q, const void* k, const void* v, int B, int H, int N, int d, float beta,
+                         void* out, float* lse, int32_t* density_out, int chunk_heads, void* scratch,
+                         size_t scratch_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || chunk_heads < 0 || std::isnan(beta)) return SOLATTN_ERR_ARG;
+  if (!scratch) return SOLATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return SOLATTN_ERR_ALIGN;
+  const int BH = B * H;
+  const int C = chunk_heads == 0 ? default_chunk_heads(BH) : (chunk_heads < BH ? chunk_heads : BH);
+  HostChunkLayout L;
+  if ((rc = host_chunk_layout(N, d, C, &L))) return rc;
+  if (scratch_bytes < SOLATTN_WORKSPACE_BYTES + 2 * L.buffer) return SOLATTN_ERR_WORKSPACE;
+  int sms = 0;
+  if ((rc = current_device_sms(&sms))) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  HostPipeline pl;
+  if (!pl.ok) return SOLATTN_ERR_CUDA;
+  char* ws = static_cast<char*>(scratch);
+  char* buf[2] = {ws + SOLATTN_WORKSPACE_BYTES, ws + SOLATTN_WORKSPACE_BYTES + L.buffer};
+  const size_t nb = (static_cast<size_t>(N) + SOLATTN_BLOCK - 1) / SOLATTN_BLOCK;
+  const size_t head_bytes = static_cast<size_t>(N) * d * 2;
+  const char* hq = static_cast<const char*>(q);
+  const char* hk = static_cast<const char*>(k);
+  const char* hv = static_cast<const char*>(v);
+  char* ho = static_cast<char*>(out);
+  const solattn_options_t opt{SOLATTN_RULE_THRESHOLD, beta, 0, 0.f, 0, {0, 0, 0}, 0};
+  auto cuda_ok = [](cudaError_t e) { return e == cudaSuccess; };
+
+  // everything earlier on the caller's stream (an earlier call on this
+  // scratch included) comes first; the status block starts clean
+  if (!cuda_ok(cudaMemsetAsync(ws, 0, SOLATTN_WORKSPACE_BYTES, s)) || !cuda_ok(cudaEventRecord(pl.start, s)) ||
+      !cuda_ok(cudaStreamWaitEvent(pl.up, pl.start, 0)) || !cuda_ok(cudaStreamWaitEvent(pl.down, pl.start, 0)))
+    return SOLATTN_ERR_CUDA;
+  const int chunks = (BH + C - 1) / C;
+  for (int i = 0; i < chunks; ++i) {
+    const int c0 = i * C, nc = (BH - c0 < C) ? BH - c0 : C;
+    char* b = buf[i & 1];
+    cudaEvent_t* in = pl.ev[0];
+    cudaEvent_t* done = pl.ev[1];
+    cudaEvent_t* back = pl.ev[2];
+    // copy in: the buffer's inputs are free once chunk i - 2 has been computed
+    if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(pl.up, done[(i - 2) & 3], 0))) return SOLATTN_ERR_CUDA;
+    const size_t bytes = head_bytes * nc, at = head_bytes * c0;
+    if (!cuda_ok(cudaMemcpyAsync(b + L.q, hq + at, bytes, cudaMemcpyHostToDevice, pl.up)) ||
+        !cuda_ok(cudaMemcpyAsync(b + L.k, hk + at, bytes, cudaMemcpyHostToDevice, pl.up)) ||
+        !cuda_ok(cudaMemcpyAsync(b + L.v, hv + at, bytes, cudaMemcpyHostToDevice, pl.up)) ||
+        !cuda_ok(cudaEventRecord(in[i & 3], pl.up)))
+      return SOLATTN_ERR_CUDA;
+    // compute: its outputs overwrite chunk i - 2's, which must have been copied back
+    if (!cuda_ok(cudaStreamWaitEvent(s, in[i & 3], 0))) return SOLATTN_ERR_CUDA;
+    if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(s, back[(i - 2) & 3], 0))) return SOLATTN_ERR_CUDA;
+    solattn_pooled_t pooled;
+    if ((rc = solattn_pooled_layout(1, nc, N, d, b + L.pooled, &pooled, nullptr))) return rc;
+    if ((rc = run_pool(b + L.q, b + L.k, b + L.v, 1, nc, N, d, nullptr, &pooled, stream))) return rc;
+    if ((rc = run_forward(b + L.q, b + L.k, b + L.v, 1, nc, N, d, &pooled, opt, true, b + L.out,
+                          lse ? reinterpret_cast<float*>(b + L.lse) : nullptr,
+                          density_out ? reinterpret_cast<int32_t*>(b + L.dens) : nullptr, ws,
+                          SOLATTN_WORKSPACE_BYTES, stream, false)))
+      return rc;
+    if (!cuda_ok(cudaEventRecord(done[i & 3], s))) return SOLATTN_ERR_CUDA;
+    // copy back
+    if (!cuda_ok(cudaStreamWaitEvent(pl.down, done[i & 3], 0)) ||
+        !cuda_ok(cudaMemcpyAsync(ho + at, b + L.out, bytes, cudaMemcpyDeviceToHost, pl.down)))
+      return SOLATTN_ERR_CUDA;
+    if (lse && !cuda_ok(cudaMemcpyAsync(lse + static_cast<size_t>(c0) * N, b + L.lse,
+                                        static_cast<size_t>(nc) * N * sizeof(float), cudaMemcpyDeviceToHost,
+                                        pl.down)))
+      return SOLATTN_ERR_CUDA;
+    if (density_out && !cuda_ok(cudaMemcpyAsync(density_out + static_cast<size_t>(c0) * nb, b + L.dens,
+                                                static_cast<size_t>(nc) * nb * sizeof(int32_t),
+                                                cudaMemcpyDeviceToHost, pl.down)))
+      return SOLATTN_ERR_CUDA;
+    if (!cuda_ok(cudaEventRecord(back[i & 3], pl.down))) return SOLATTN_ERR_CUDA;
+  }
+  // the results are on the host once the caller's stream has passed this point
+  if (!cuda_ok(cudaStreamWaitEvent(s, pl.ev[2][(chunks - 1) & 3], 0))) return SOLATTN_ERR_CUDA;
+  return SOLATTN_OK;
 }
 
 }  // extern "C"

@@ -264,6 +264,39 @@ int solattn_forward_noalloc(const void* q, const void* k, const void* v, int B, 
  */
 int solattn_noalloc_status(void* stream);
 
+/*
+ * End-to-end forward on HOST buffers (no counterpart on the pages): the
+ * computation of solattn_pool + solattn_forward (threshold rule, block-level
+ * correction) for q, k, v in host memory, with out, lse and density_out
+ * written to host memory. Layouts are the contiguous ones of solattn_forward;
+ * lse and density_out may be NULL.
+ *
+ * The B*H (batch, head) pairs are independent (every statistic and every
+ * kept set is per pair), so they go through the device in chunks of
+ * chunk_heads consecutive pairs (0 = about B*H / 16, at least 1): while chunk i
+ * is pooled and attended on `stream`, chunk i + 1 is copied to the device and
+ * chunk i - 1's results are copied back, on two streams of the call's own.
+ * Host buffers must be page-locked (cudaHostAlloc / cudaHostRegister) for the
+ * copies to overlap the computation; pageable memory gives the same results
+ * with the copies serialised by the CUDA runtime.
+ *
+ * scratch: device memory of at least solattn_host_scratch_bytes(B, H, N, d,
+ * chunk_heads) bytes, 256-byte aligned, owned by the caller and used by one
+ * call at a time (two chunk buffers of inputs, outputs and pooled statistics;
+ * its first SOLATTN_WORKSPACE_BYTES are the workspace, so
+ * solattn_status(scratch, stream) reports the call's device status: the first
+ * error of any chunk). The call only enqueues work; the results are in host
+ * memory once `stream` has completed (the call makes `stream` wait for the
+ * last copy back). Errors: as for solattn_forward, plus SOLATTN_ERR_ARG for a
+ * null host buffer, a negative chunk_heads or a NaN beta, and
+ * SOLATTN_ERR_WORKSPACE for a missing or short scratch; nothing is enqueued
+ * when the arguments are rejected.
+ */
+int solattn_host_scratch_bytes(int B, int H, int N, int d, int chunk_heads, size_t* bytes);
+int solattn_forward_host(const void* q, const void* k, const void* v, int B, int H, int N, int d, float beta,
+                         void* out, float* lse, int32_t* density_out, int chunk_heads, void* scratch,
+                         size_t scratch_bytes, void* stream);
+
 /* Static description of a status code. */
 const char* solattn_strerror(int code);
 

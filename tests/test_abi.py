@@ -146,7 +146,7 @@ def test_noalloc_path_names_no_allocating_call():
     """The allocation-free entry point and its helpers call no device
     allocator (checked on the source of the noalloc section of api.cu)."""
     src = open(os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", "api.cu")).read()
-    section = src[src.index("Allocation-free forward"):]
+    section = src[src.index("Allocation-free forward"):src.index("End-to-end forward on host buffers")]
     code = re.sub(r"//[^\n]*", "", section)
     for name in ("cudaMalloc", "cudaMallocAsync", "cudaMallocManaged", "cudaFree", "malloc(", "new ", "torch"):
         assert name not in code, name
@@ -175,3 +175,38 @@ def test_dense_rejects_non_contiguous_views():
     x = torch.zeros((1, 4, 2, 64), dtype=torch.bfloat16).permute(0, 2, 1, 3)  # [B, N, H, d] seen as [B, H, N, d]
     with pytest.raises(ValueError, match="contiguous"):
         sa.dense(x, x, x)
+
+
+def test_host_scratch_sizes(L):
+    """Two chunk buffers (q, k, v, out, lse, density and the chunk's pooled
+    statistics, each 256-byte aligned) after the workspace."""
+    B, H, N, d = 1, 40, 75600, 128
+    nb = math.ceil(N / 64)
+    r = lambda x: (x + 255) // 256 * 256
+    for chunk, C in ((0, 3), (5, 5), (100, 40)):
+        n, p = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        assert L.solattn_host_scratch_bytes(B, H, N, d, chunk, ctypes.byref(n)) == 0
+        assert L.solattn_pooled_layout(1, C, N, d, None, None, ctypes.byref(p)) == 0
+        buf = 4 * r(C * N * d * 2) + r(C * N * 4) + r(C * nb * 4) + r(p.value)
+        assert n.value == _lib.WORKSPACE_BYTES + 2 * buf, chunk
+    assert L.solattn_host_scratch_bytes(B, H, N, d, -1, ctypes.byref(n)) == _lib.ERR_ARG
+    assert L.solattn_host_scratch_bytes(B, H, N, 80, 0, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED
+    assert L.solattn_host_scratch_bytes(B, H, N, d, 0, None) == _lib.ERR_ARG
+
+
+def test_forward_host_argument_errors(L):
+    h = ctypes.create_string_buffer(64)
+    p = ctypes.cast(h, ctypes.c_void_p)
+    scratch = ctypes.c_void_p(0x10000000)
+    f = ctypes.c_float
+    args = lambda q=p, out=p, beta=0.5, chunk=0, sc=scratch, n=1 << 30: (
+        q, p, p, 1, 2, 256, 64, f(beta), out, None, None, chunk, sc, n, None)
+    assert L.solattn_forward_host(*args(q=None)) == _lib.ERR_ARG
+    assert L.solattn_forward_host(*args(out=None)) == _lib.ERR_ARG
+    assert L.solattn_forward_host(*args(beta=float("nan"))) == _lib.ERR_ARG
+    assert L.solattn_forward_host(*args(chunk=-1)) == _lib.ERR_ARG
+    assert L.solattn_forward_host(*args(sc=None)) == _lib.ERR_WORKSPACE
+    assert L.solattn_forward_host(*args(sc=ctypes.c_void_p(0x10000010))) == _lib.ERR_ALIGN
+    assert L.solattn_forward_host(*args(n=1024)) == _lib.ERR_WORKSPACE
+    assert L.solattn_forward_host(p, p, p, 1, 2, 256, 80, f(0.5), p, None, None, 0, scratch, 1 << 30,
+                                  None) == _lib.ERR_UNSUPPORTED
