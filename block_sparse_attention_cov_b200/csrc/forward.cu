@@ -470,13 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < TT && ok; ++t) {
           const uint32_t gt = gtile + t;
           const int nb = ut.halves(t, P.NB);
-          if (!warp_wait(&sm.p_full[gt % 3], (gt / 3) & 1, abort_flag, st, kSitePFull, u)) { ok = false; break; }
+          // V first: it has normally landed long before P, so once P is
+          // stored only the issue remains
           uint32_t stv[2];
           for (int h = 0; h < nb && ok; ++h) {
             const uint32_t gv = gblk + ut.vblock(t, h);
             stv[h] = gv % VS;
             ok = warp_wait(&sm.v_full[stv[h]], (gv / VS) & 1, abort_flag, st, kSiteVFull, u);
           }
+          if (ok) ok = warp_wait(&sm.p_full[gt % 3], (gt / 3) & 1, abort_flag, st, kSitePFull, u);
           if (!ok) break;
           tc_fence_after();
           if (elect_one()) {
