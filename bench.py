@@ -12,8 +12,10 @@ heads, d = 128, beta calibrated for a 15 % mean kept-block density.
 Prints one JSON line. value = kept-block TFLOP/s of the whole step (kept-block
 FLOPs = 4 d n_i n_j summed over kept (i, j) pairs), whole job over all ranks.
 Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
-GPU (heads are independent; no collective on the data path); timing is the max
-over ranks.
+GPU (heads are independent; no collective on the data path; weak scaling), or
+with --shard heads its contiguous share of the (batch, head) pairs (strong
+scaling, the survey's head partition); timing is the max over ranks and value
+counts every rank's work.
 
 e2e = the same step through solattn_forward_host: q, k, v in pinned host
 memory, out, lse and density back to pinned host memory, the copies inside the
@@ -343,6 +345,23 @@ def job_value(flops_per_rank, ms, world):
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
+def sum_over_ranks(value, world, device):
+    """Sum of one per-rank number over all ranks; identity for one rank."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def head_slice(B, H, rank, world):
+    """(b, h) pairs of this rank when the B*H independent pairs are split over
+    the ranks: contiguous, balanced (sizes differ by at most one), every pair
+    on exactly one rank."""
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    lo, hi = len(pairs) * rank // world, len(pairs) * (rank + 1) // world
+    return pairs[lo:hi]
+
+
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     """The oracle as it stands (fp32 working precision, multithreaded BLAS) on
@@ -397,7 +416,17 @@ def run_ours(args, rank, world, local_rank):
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
     peaks = load_peaks()
 
-    q_h, k_h, v_h = make_qkv(wl, seed=0)
+    sharded = args.shard == "heads" and world > 1
+    if sharded:
+        # strong scaling: this rank's contiguous share of the (b, h) pairs,
+        # attended as one batch of heads (the pairs are independent)
+        mine = head_slice(B, H, rank, world)
+        if not mine:
+            raise SystemExit(f"--shard heads needs at least {world} (batch, head) pairs")
+        q_h, k_h, v_h = make_qkv(wl, seed=0, heads=mine)
+        B, H = 1, len(mine)
+    else:
+        q_h, k_h, v_h = make_qkv(wl, seed=0)
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     stream = torch.cuda.current_stream()
     ws = sa.workspace(dev)
@@ -427,6 +456,11 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {sa.status(ws)} after warm-up")
     kflops = kept_flops(stats, dens, beta, N, d, args.rule, args.n_forced)
     mean_density = float(dens.double().mean().item()) / nb
+    # work of the whole job: every rank's own share (sharded) or copy (replicas)
+    job_kflops = sum_over_ranks(kflops, world, dev) if sharded else world * kflops
+    # the union of each unit's two kept sets: what the tensor pipe multiplies
+    uflops = union_flops(stats, beta, N, d, args.n_forced) if args.rule == "threshold" else None
+    job_uflops = None if uflops is None else (sum_over_ranks(uflops, world, dev) if sharded else world * uflops)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -507,7 +541,7 @@ def run_ours(args, rank, world, local_rank):
         (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp))
         d2h = sum(x.numel() * x.element_size() for x in (out_h, lse_h, dens_h))
-        e2e = {"value": job_value(kflops, e2e_ms, world), "unit": UNIT,
+        e2e = {"value": job_kflops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "path": "solattn_forward_host: pinned host buffers, head chunks copied in / attended / "
                        "copied back on three streams"}
@@ -516,7 +550,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
 
-    fwd_tflops = kflops / (fwd_ms * 1e-3) / 1e12
+    fwd_tflops = job_kflops / world / (fwd_ms * 1e-3) / 1e12  # per GPU
     # The timed loop runs the kernel back to back; once it lasts a second or
     # more the GPU sits at its power cap, so the sustained GEMM figure (taken
     # the same way) is the like-for-like denominator, else the burst one.
@@ -529,28 +563,28 @@ def run_ours(args, rank, world, local_rank):
     cpu, parity = None, None
     if not args.skip_cpu and world == 1 and args.rule == "threshold" and not args.n_forced:
         cpu, parity = cpu_baseline_leg(q_h, k_h, v_h, beta, dens.cpu().numpy())
-    uflops = union_flops(stats, beta, N, d, args.n_forced) if args.rule == "threshold" else None
     line = {
         "metric": METRIC,
-        "value": job_value(kflops, ms_step, world),
+        "value": job_kflops / (ms_step * 1e-3) / 1e12,
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; bf16)",
         "config": {
-            "workload": args.workload, "B": B, "H": H, "N": N, "d": d, "grid": list(wl.grid), "beta": beta,
+            "workload": args.workload, "B": wl.B, "H": wl.H, "N": N, "d": d, "grid": list(wl.grid), "beta": beta,
             "rule": args.rule, **({"topk": args.topk} if args.rule == "topk" else {}),
             **({"topp": args.topp} if args.rule == "topp" else {}),
             **({"n_forced": args.n_forced} if args.n_forced else {}),
             **({"correction": args.correction} if args.correction != "block" else {}),
-            "mean_density": mean_density, "global_batch": B * world, "seq_len": N,
-            "parallelism": f"heads-independent replicas x{world}",
+            "mean_density": mean_density, "global_batch": 1 if sharded else B * world, "seq_len": N,
+            "parallelism": (f"(batch, head) pairs sharded over {world} ranks, {H} on this rank" if sharded
+                            else f"heads-independent replicas x{world}"),
             "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no explicit flush" % (B * H * N * d * 2 / 1e6),
         },
         "fwd_ms": fwd_ms,
@@ -562,9 +596,9 @@ def run_ours(args, rank, world, local_rank):
         "pool_frac_hbm": pool_gbs / peaks["hbm_gbs"],
         "dense_ms": dense_ms,
         "speedup_vs_dense": (dense_ms / fwd_ms) if dense_ms else None,
-        "kept_tflop_per_step": kflops / 1e12,
-        "union_tflop_per_step": None if uflops is None else uflops / 1e12,
-        "pair_efficiency": None if uflops is None else kflops / uflops,
+        "kept_tflop_per_step": job_kflops / 1e12,
+        "union_tflop_per_step": None if uflops is None else job_uflops / 1e12,
+        "pair_efficiency": None if uflops is None else job_kflops / job_uflops,
         "density": density_stats(dens, nb),
         "near_ties": None if parity is None else parity["near_ties"],
         "density_mismatch_rows": None if parity is None else parity["density_mismatch_rows"],
@@ -698,6 +732,10 @@ def main():
     ap.add_argument("--n-forced", type=int, default=0, help="leading key blocks always kept")
     ap.add_argument("--correction", choices=["block", "token"], default="block",
                     help="skipped-block correction: block-level proxy score (the method) or per token")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="multi-GPU layout: every rank runs the whole workload (weak scaling), or the (batch, "
+                         "head) pairs are split over the ranks (strong scaling); no collective on the data path "
+                         "either way")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-dense", action="store_true")

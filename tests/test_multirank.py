@@ -30,7 +30,8 @@ def _worker(rank, world, port, out):
         import bench
 
         got = bench.max_over_ranks([10.0 + rank, 5.0 - rank], world, "cpu")
-        out.put((rank, got, bench.job_value(1e12, got[0], world)))
+        total = bench.sum_over_ranks(1e12 * (rank + 1), world, "cpu")
+        out.put((rank, got, bench.job_value(1e12, got[0], world), total))
     finally:
         dist.destroy_process_group()
 
@@ -46,9 +47,24 @@ def test_max_over_ranks_and_job_value_with_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, got, value in res:
+    for rank, got, value, total in res:
         assert got == [11.0, 5.0]  # slowest rank per entry
         assert value == pytest.approx(2 * 1e12 / 11e-3 / 1e12)
+        assert total == pytest.approx(3e12)  # every rank's own work, summed on every rank
+
+
+@pytest.mark.parametrize("B,H,world", [(1, 40, 8), (1, 40, 3), (2, 3, 4), (1, 24, 24), (3, 5, 2)])
+def test_head_slices_cover_every_pair_once_and_balance(B, H, world):
+    """The head-sharded layout: the ranks' contiguous shares of the (b, h)
+    pairs are disjoint, cover all B*H pairs in order, and differ in size by at
+    most one."""
+    import bench
+
+    slices = [bench.head_slice(B, H, r, world) for r in range(world)]
+    flat = [p for sl in slices for p in sl]
+    assert flat == [(b, h) for b in range(B) for h in range(H)]
+    sizes = [len(sl) for sl in slices]
+    assert max(sizes) - min(sizes) <= 1
 
 
 def test_reference_arm_prints_once_from_rank_zero_under_torchrun():
