@@ -255,9 +255,12 @@ def row_kept_flops(mask, N, d):
     return 4.0 * d * n * (mask.astype(np.float64) @ n)
 
 
-def oracle_head_sample(q, k, v, beta, head_pos, head_id, seed=0):
+def oracle_head_sample(q, k, v, beta, head_pos, head_id, seed=0, out_gpu=None, lse_gpu=None):
     """The oracle (fp32 working precision, multithreaded BLAS) on the stratified
-    sample of one head. Returns (seconds, kept FLOPs of the sample)."""
+    sample of one head. Returns (seconds, kept FLOPs of the sample, error sums):
+    with the GPU's out / lse of this head ([N, d], [N] numpy), the squared
+    error and squared norm of out over the sampled rows, its max abs error and
+    the max lse error (outside the timed call)."""
     from oracle import solattn_oracle as orc
 
     N, d = q.shape[2], q.shape[3]
@@ -265,10 +268,16 @@ def oracle_head_sample(q, k, v, beta, head_pos, head_id, seed=0):
     rows = sample_rows(nb, head_id, seed)
     qq, kk, vv = (x[0, head_pos].float().numpy() for x in (q, k, v))
     t0 = time.perf_counter()
-    orc.attend(qq, kk, vv, beta, rows=rows, dtype=np.float32)
+    o, l, _ = orc.attend(qq, kk, vv, beta, rows=rows, dtype=np.float32)
     secs = time.perf_counter() - t0
     r = orc.route(qq, kk, beta, dtype=np.float32)
-    return secs, float(row_kept_flops(r["mask"], N, d)[rows].sum())
+    errs = None
+    if out_gpu is not None:
+        tok = np.concatenate([np.arange(64 * i, min(64 * i + 64, N)) for i in rows])
+        e = out_gpu[tok].astype(np.float64) - o[tok].astype(np.float64)
+        errs = (float((e * e).sum()), float((o[tok].astype(np.float64) ** 2).sum()), float(np.abs(e).max()),
+                float(np.abs(lse_gpu[tok].astype(np.float64) - l[tok]).max()))
+    return secs, float(row_kept_flops(r["mask"], N, d)[rows].sum()), errs
 
 
 def routing_oracle(q, k, beta, dens_gpu):
@@ -292,7 +301,7 @@ def routing_oracle(q, k, beta, dens_gpu):
     return secs, ties, bad, np.stack(flops)
 
 
-def cpu_baseline_leg(q, k, v, beta, dens_gpu, seed=0):
+def cpu_baseline_leg(q, k, v, beta, dens_gpu, seed=0, out_gpu=None, lse_gpu=None):
     """CPU baseline as the oracle stands: fp32 multithreaded BLAS on the
     stratified sample of every head (first, last, 30 random query blocks),
     with the full forward's CPU time extrapolated from it by kept FLOPs; the
@@ -304,10 +313,16 @@ def cpu_baseline_leg(q, k, v, beta, dens_gpu, seed=0):
     nb = math.ceil(N / 64)
     r_secs, ties, bad, row_flops = routing_oracle(q, k, beta, dens_gpu)
     s_secs, s_flops = 0.0, 0.0
+    err2 = ref2 = emax = lmax = 0.0
     for h in range(H):
-        t, f = oracle_head_sample(q, k, v, beta, h, h, seed)
+        t, f, errs = oracle_head_sample(q, k, v, beta, h, h, seed,
+                                        None if out_gpu is None else out_gpu[0, h],
+                                        None if lse_gpu is None else lse_gpu[0, h])
         s_secs += t
         s_flops += f
+        if errs is not None:
+            err2, ref2 = err2 + errs[0], ref2 + errs[1]
+            emax, lmax = max(emax, errs[2]), max(lmax, errs[3])
     total_flops = float(row_flops.sum())
     full = {}
     for name, wl_beta in (("tiny", 1.0), ("mid", 1.0)):
@@ -327,7 +342,10 @@ def cpu_baseline_leg(q, k, v, beta, dens_gpu, seed=0):
         "full_forward_seconds_extrapolated": s_secs * total_flops / s_flops,
         "routing_oracle_seconds_all_blocks": r_secs,
         "full_runs": full,
-    }, {"near_ties": ties, "density_mismatch_rows": bad, "rows": int(H * nb)}
+    }, {"near_ties": ties, "density_mismatch_rows": bad, "rows": int(H * nb),
+        "output_error": None if out_gpu is None else {
+            "rel_l2": math.sqrt(err2 / ref2), "max_abs": emax, "max_lse": lmax,
+            "against": f"oracle fp32 on the stratified sample ({H} heads x {SAMPLE_BLOCKS} query blocks)"}}
 
 
 def max_over_ranks(values, world, device):
@@ -378,7 +396,7 @@ def run_reference(args, rank, world):
     times, flops = [], 0.0
     for step in range(args.warmup + args.steps):
         h = step % wl.H
-        t, f = oracle_head_sample(q, k, v, beta, pos[h], h)
+        t, f, _ = oracle_head_sample(q, k, v, beta, pos[h], h)
         if step >= args.warmup:
             times.append(t)
             flops += f
@@ -562,7 +580,8 @@ def run_ours(args, rank, world, local_rank):
     pool_gbs = pbytes / (pool_ms * 1e-3) / 1e9
     cpu, parity = None, None
     if not args.skip_cpu and world == 1 and args.rule == "threshold" and not args.n_forced:
-        cpu, parity = cpu_baseline_leg(q_h, k_h, v_h, beta, dens.cpu().numpy())
+        cpu, parity = cpu_baseline_leg(q_h, k_h, v_h, beta, dens.cpu().numpy(), out_gpu=out.float().cpu().numpy(),
+                                       lse_gpu=lse.cpu().numpy())
     line = {
         "metric": METRIC,
         "value": job_kflops / (ms_step * 1e-3) / 1e12,
@@ -602,6 +621,7 @@ def run_ours(args, rank, world, local_rank):
         "density": density_stats(dens, nb),
         "near_ties": None if parity is None else parity["near_ties"],
         "density_mismatch_rows": None if parity is None else parity["density_mismatch_rows"],
+        "output_error": None if parity is None else parity["output_error"],
         "roofline": {
             "bound": "tensor",
             "achieved": fwd_tflops,

@@ -60,3 +60,24 @@ def test_density_stats():
     st = bench.density_stats(dens, 8)
     assert st["mean"] == pytest.approx(2.5 / 8) and st["min"] == 1 / 8 and st["max"] == 4 / 8
     assert st["p50"] == pytest.approx(2.5 / 8)
+
+
+def test_oracle_head_sample_reports_output_error():
+    """The bench line's output_error: against the fp32 oracle on the sampled
+    rows, an exact (fp64 oracle) output gives a tiny error and a perturbed one
+    is caught at the perturbation's size."""
+    import numpy as np
+
+    import bench
+    from block_sparse_attention_cov_b200.inputs import Workload, make_qkv
+    from oracle import solattn_oracle as orc
+
+    wl = Workload("s", 1, 1, 64, (1, 1, 64 * 40))
+    q, k, v = make_qkv(wl, seed=3)
+    out64, lse64, _ = orc.attend(*(x[0, 0].double().numpy() for x in (q, k, v)), 0.5)
+    _, _, errs = bench.oracle_head_sample(q, k, v, 0.5, 0, 0, out_gpu=out64, lse_gpu=lse64)
+    assert errs[0] / errs[1] < 1e-10 and errs[2] < 1e-5 and errs[3] < 1e-5
+    bad = out64.copy()
+    bad[0, 0] += 0.25  # row 0 belongs to the first block, always sampled
+    _, _, errs = bench.oracle_head_sample(q, k, v, 0.5, 0, 0, out_gpu=bad, lse_gpu=lse64)
+    assert abs(errs[2] - 0.25) < 1e-4
