@@ -578,6 +578,10 @@ def run_ours(args, rank, world, local_rank):
         peak_tc, peak_kind = peaks["bf16_tflops"], " (bf16 burst)"
     pbytes = pool_bytes(B, H, N, d)
     pool_gbs = pbytes / (pool_ms * 1e-3) / 1e9
+    # the threshold rule with the block-level correction runs on the two-group
+    # kernel (whose ncu traffic record bench reports); the other variants on
+    # the one-unit kernel
+    two_group = args.rule == "threshold" and args.correction == "block"
     cpu, parity = None, None
     if not args.skip_cpu and world == 1 and args.rule == "threshold" and not args.n_forced:
         cpu, parity = cpu_baseline_leg(q_h, k_h, v_h, beta, dens.cpu().numpy(), out_gpu=out.float().cpu().numpy(),
@@ -628,8 +632,9 @@ def run_ours(args, rank, world, local_rank):
             "peak": peak_tc,
             "unit": "TFLOP/s",
             "frac": fwd_tflops / peak_tc,
-            "traffic": fwd_traffic(B * H),
-            "kernel": "solattn_fwd_pp_kernel (fused forward)",
+            "traffic": fwd_traffic(B * H) if two_group else None,
+            "kernel": "solattn_fwd_pp_kernel (fused forward)" if two_group
+                      else "solattn_fwd_kernel (fused forward, one-unit kernel)",
             "peak_source": peaks["source"] + peak_kind,
         },
         "pool_roofline": {
