@@ -205,3 +205,35 @@ def test_output_in_own_and_external_mask_modes(name, wl, betas, heads, rows):
               f"external mask rel-L2 {e_ext[0]:.2e} max {e_ext[1]:.2e} lse {e_ext[2]:.2e}")
         for e in (e_own, e_ext):
             assert e[0] <= 1e-2 and e[1] <= 2e-2 and e[2] <= 1e-3, (name, beta, e)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_maximum_sequence_length(d):
+    """N = 262,144 tokens, the largest the library accepts (4,096 key blocks:
+    the routing warps' bitmap capacity and, for top-k / top-p, the proxy rows
+    held in shared memory): the kept mask bit-exact against the oracle (near
+    ties counted), the output on 15 query blocks (first, middle, last two and
+    11 seeded random) within the usual tolerances, and the top-k mask at the
+    same size."""
+    wl = _wl(1, 1, d, 262144)
+    q, k, v = make_qkv(wl, seed=7)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    beta = 1.0
+    out, lse, dens, mask, stats = forward_with_routing(qd, kd, vd, beta)
+    _check_threshold(q, k, beta, mask, stats, dens.cpu().numpy(), f"N=262144 d={d}")
+    nb = 4096
+    rng = np.random.default_rng(d)
+    rows = sorted({0, 2047, nb - 2, nb - 1, *rng.choice(np.arange(1, nb - 2), 11, replace=False).tolist()})
+    own = orc.forward(q, k, v, beta, rows=rows)
+    tok = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in rows])
+    e = _out_errors(out.float().cpu().numpy()[:, :, tok], lse.cpu().numpy()[:, :, tok], own[0][:, :, tok],
+                    own[1][:, :, tok])
+    print(f"N=262144 d={d}: out rel-L2 {e[0]:.2e} max {e[1]:.2e} lse {e[2]:.2e}")
+    assert e[0] <= 1e-2 and e[1] <= 2e-2 and e[2] <= 1e-3, e
+    _, _, dk, mk, _ = forward_with_routing(qd, kd, vd, 0.0, rule="topk", topk=600)
+    r = orc.route_rule(q[0, 0].double().numpy(), k[0, 0].double().numpy(), "topk", 600, 0)
+    near = _rule_near(r, "topk", 600, wl.N)
+    diff = mk[0, 0] != r["mask"]
+    assert not (diff & ~near).any(), np.argwhere(diff & ~near)[:5]
+    assert (dk.cpu().numpy()[0, 0] == mk[0, 0].sum(-1)).all()
+    print(f"N=262144 d={d} top-k 600: {int(near.sum())} near ties, {int(diff.sum())} flipped")
