@@ -110,9 +110,10 @@ def test_kept_mask_on_the_large_workloads(name, heads):
 
 def _rule_near(r, rule, param, N):
     """Per (i, j): True where the oracle's decision is a near tie at the rule's
-    cut (top-k: a score within 1e-4 of the k-th largest; top-p: the whole row
-    when its cumulative mass crosses p within 1e-4 of the total or the cut
-    value is tied)."""
+    cut (top-k: a score within 1e-4 of the k-th largest; top-p: the blocks
+    whose membership depends on where the cumulative mass, in descending score
+    order, crosses p within 1e-4 of the total (from the first position of that
+    band to the one after its last), and scores within 1e-4 of the cut value)."""
     shat = r["shat"]
     nb = shat.shape[1]
     near = np.zeros(shat.shape, bool)
@@ -127,8 +128,9 @@ def _rule_near(r, rule, param, N):
             cum = np.cumsum(w) - param * w.sum()
             kp = min(int(np.searchsorted(cum, 0.0, side="left")), nb - 1)
             vstar = shat[i, order[kp]]
-            if (np.abs(cum) <= TIE * w.sum()).any():
-                near[i] = True
+            band = np.nonzero(np.abs(cum) <= TIE * w.sum())[0]
+            if len(band):
+                near[i, order[band.min():band.max() + 2]] = True
             near[i] |= np.abs(shat[i] - vstar) <= TIE
     elif rule == "threshold":
         near = np.abs(shat - r["tau"][:, None]) <= TIE
@@ -213,8 +215,8 @@ def test_maximum_sequence_length(d):
     the routing warps' bitmap capacity and, for top-k / top-p, the proxy rows
     held in shared memory): the kept mask bit-exact against the oracle (near
     ties counted), the output on 15 query blocks (first, middle, last two and
-    11 seeded random) within the usual tolerances, and the top-k mask at the
-    same size."""
+    11 seeded random) within the usual tolerances, and the top-k and top-p
+    masks at the same size."""
     wl = _wl(1, 1, d, 262144)
     q, k, v = make_qkv(wl, seed=7)
     qd, kd, vd = (x.cuda() for x in (q, k, v))
@@ -237,3 +239,10 @@ def test_maximum_sequence_length(d):
     assert not (diff & ~near).any(), np.argwhere(diff & ~near)[:5]
     assert (dk.cpu().numpy()[0, 0] == mk[0, 0].sum(-1)).all()
     print(f"N=262144 d={d} top-k 600: {int(near.sum())} near ties, {int(diff.sum())} flipped")
+    _, _, dp, mp, _ = forward_with_routing(qd, kd, vd, 0.0, rule="topp", topp=0.5)
+    r = orc.route_rule(q[0, 0].double().numpy(), k[0, 0].double().numpy(), "topp", 0.5, 0)
+    near = _rule_near(r, "topp", 0.5, wl.N)
+    diff = mp[0, 0] != r["mask"]
+    assert not (diff & ~near).any(), np.argwhere(diff & ~near)[:5]
+    assert (dp.cpu().numpy()[0, 0] == mp[0, 0].sum(-1)).all()
+    print(f"N=262144 d={d} top-p 0.5: {int(near.sum())} near ties, {int(diff.sum())} flipped")

@@ -194,3 +194,65 @@ def test_full_size_wan_routing_exact_and_sampled_rows():
             for i in rows:
                 m[i * 64:min(wl.N, i * 64 + 64)] = True
             _check_out(out[0, h], lse[0, h], oo, lo, m)
+
+
+def test_dense_path_at_the_maximum_length():
+    """solattn_dense at N = 262,144 (4,096 key blocks, every tile of every
+    unit) on 12 query blocks against the oracle's dense attention."""
+    wl = _wl(1, 1, 128, 262144)
+    q, k, v = make_qkv(wl, seed=8)
+    qd, kd, vd = _dev(q, k, v)
+    ws = sa.workspace()
+    od, ld = sa.dense(qd, kd, vd, ws=ws)
+    assert sa.status(ws) == 0
+    nb = 4096
+    rng = np.random.default_rng(1)
+    rows = sorted({0, 2047, nb - 1, *rng.choice(np.arange(1, nb - 1), 9, replace=False).tolist()})
+    tok = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in rows])
+    qq, kk, vv = (x[0, 0].double().numpy() for x in (q, k, v))
+    s = 1.0 / math.sqrt(128)
+    sc = s * (qq[tok] @ kk.T)
+    m = sc.max(axis=1, keepdims=True)
+    e = np.exp(sc - m)
+    den = e.sum(axis=1)
+    out_o = np.full((wl.N, 128), np.nan)
+    lse_o = np.full((wl.N,), np.nan)
+    out_o[tok] = (e @ vv) / den[:, None]
+    lse_o[tok] = m[:, 0] + np.log(den)
+    keep = np.zeros(wl.N, bool)
+    keep[tok] = True
+    _check_out(od[0, 0], ld[0, 0], out_o, lse_o, keep)
+
+
+def test_many_heads_over_two_batches():
+    """Two batches of 24 heads at 16,384 tokens (a unit queue of 6,144 units
+    over the persistent CTAs, head-major across the batch boundary): every
+    block's kept count against the routing oracle and the output of sampled
+    query blocks in a head of each batch."""
+    import json
+    import os
+
+    wl = Workload("b2h24", 2, 24, 128, (5, 45, 80), 16384)
+    with open(os.path.join(os.path.dirname(__file__), "golden", "calibrated_beta.json")) as f:
+        beta = json.load(f)["sweep_16k"]["targets"]["0.15"]["beta"]
+    q, k, v = make_qkv(wl, seed=9)
+    qd, kd, vd = _dev(q, k, v)
+    st = sa.pool(qd, kd, vd)
+    ws = sa.workspace()
+    out, lse, dens = sa.forward(qd, kd, vd, st, beta, ws=ws)
+    assert sa.status(ws) == 0
+    dens = dens.cpu().numpy()
+    nb = 256
+    for b in range(2):
+        for h in range(24):
+            qq, kk = q[b, h].double().numpy(), k[b, h].double().numpy()
+            r = orc.route(qq, kk, beta)
+            ties = (np.abs(r["shat"] - r["tau"][:, None]) <= TIE).sum(-1)
+            _check_density(dens[b, h], r["density"], ties)
+            if h == 23 - 11 * b:
+                rows = [0, 1, 100, nb - 1]
+                oo, lo, _ = orc.attend(qq, kk, v[b, h].double().numpy(), beta, rows=rows)
+                m = np.zeros(wl.N, bool)
+                for i in rows:
+                    m[i * 64:i * 64 + 64] = True
+                _check_out(out[b, h], lse[b, h], oo, lo, m)
