@@ -129,18 +129,29 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- traffic record
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "solattn_fwd_pp_kernel.traffic.txt")
-FWD_SOURCE = os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", "forward_pp.cu")
+FWD_SOURCES = [os.path.join(ROOT, "block_sparse_attention_cov_b200", "csrc", f)
+               for f in ("forward_pp.cu", "fwd_common.cuh", "ptx.cuh")]
+
+
+def fwd_source_digest():
+    """sha256 over the two-group kernel's sources (the kernel and the headers
+    it compiles in), in a fixed order."""
+    h = hashlib.sha256()
+    for f in FWD_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
 
 
 def fwd_traffic(heads):
     """DRAM bytes (read + write) of one forward launch at `heads` heads, from the
     committed ncu record of a small capture scaled by the units processed; None
     when the record is missing or was taken on another version of the kernel
-    source (its sha256 no longer matches)."""
+    source (its sha256 over forward_pp.cu, fwd_common.cuh and ptx.cuh no
+    longer matches)."""
     try:
         rec = dict(ln.split(":", 1) for ln in open(TRAFFIC_RECORD).read().splitlines() if ":" in ln)
         rec = {k.strip(): v.strip() for k, v in rec.items()}
-        digest = hashlib.sha256(open(FWD_SOURCE, "rb").read()).hexdigest()
+        digest = fwd_source_digest()
         if rec.get("source_sha256") != digest:
             return None
         per_head = (float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])) / float(rec["heads"])

@@ -28,7 +28,7 @@
 // store) overlap the exponentials of the next.
 //
 // Both groups feed the one O, so all P of a row share one reference max m.
-// It only moves up, and lazily (when a tile's max exceeds it by more than 8 in
+// It only moves up, and lazily (when a tile's max exceeds it by more than 16 in
 // log2 units), and it is kept integral, so every rescale is an exact power of
 // two. A group computes a tile's P with the reference it last knew, then
 // receives the reference the other group settled for the previous tile (a

@@ -26,7 +26,7 @@ constexpr int kNbMax = 4096;  // key blocks per head supported
 constexpr int kChunk = 16;    // pooled key blocks per routing chunk (4 per routing warp)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleSlack = 8.0f;  // log2 units a row max may grow before O is rescaled
+constexpr float kRescaleSlack = 16.0f;  // log2 units a row max may grow before O is rescaled
 
 // Wait-site ids reported in the status word when a bounded wait gives up.
 enum : uint32_t {
