@@ -47,7 +47,7 @@ def pooled(L, q, k, v):
     return buf, st
 
 
-def forward_with_routing(q, k, v, beta=0.0, rule="threshold", topk=0, topp=0.0, n_forced=0):
+def forward_with_routing(q, k, v, beta=0.0, rule="threshold", topk=0, topp=0.0, n_forced=0, correction="block"):
     """One forward through the hook build with the routing copy switched on.
 
     Returns (out, lse, density, mask, stats): mask [B, H, N_b, N_b] bool (the
@@ -68,7 +68,7 @@ def forward_with_routing(q, k, v, beta=0.0, rule="threshold", topk=0, topp=0.0, 
     try:
         rules = {"threshold": _lib.RULE_THRESHOLD, "topk": _lib.RULE_TOPK, "topp": _lib.RULE_TOPP}
         opts = _lib.OptionsStruct(rules[rule], float(beta), int(topk), float(topp), int(n_forced),
-                                  _lib.StridesStruct(0, 0, 0), 0)
+                                  _lib.StridesStruct(0, 0, 0), 1 if correction == "token" else 0)
         rc = L.solattn_forward_ex(_p(q), _p(k), _p(v), B, H, N, d, ctypes.byref(st), ctypes.byref(opts), _p(out),
                                   _p(lse), _p(dens), _p(ws), ws.numel(), stream)
         assert rc == 0, _lib.strerror(rc)

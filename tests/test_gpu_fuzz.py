@@ -60,3 +60,55 @@ def test_random_shapes_match_oracle(seed):
     print(f"B={B} H={H} d={d} N={N} beta={beta:.3f}: rel-L2 {rel:.2e} max {np.abs(err).max():.2e} "
           f"lse {dl:.2e} near ties {int(near.sum())} flipped {int(diff.sum())}")
     assert rel <= 1e-2 and np.abs(err).max() <= 2e-2 and dl <= 1e-3
+
+
+def _case_rules(seed):
+    rng = np.random.default_rng(2000 + seed)
+    B, H = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+    d = int(rng.choice([64, 128]))
+    N = int(rng.integers(2, 4000))
+    nb = math.ceil(N / 64)
+    rule = ["topk", "topp", "threshold", "threshold"][seed % 4]
+    param = {"topk": int(rng.integers(0, nb + 2)), "topp": float(rng.uniform(0.0, 1.05)),
+             "threshold": float(rng.normal(0.5, 0.6))}[rule]
+    n_forced = int(rng.integers(0, 4)) if seed % 3 == 0 else 0
+    correction = "token" if seed % 4 == 3 else "block"
+    return B, H, d, N, rule, param, n_forced, correction
+
+
+@pytest.mark.parametrize("seed", list(range(12)))
+def test_random_shapes_other_rules_and_token_correction(seed):
+    """Top-k (k from 0 past N_b), top-p (p from 0 past 1), the threshold with
+    forced leading blocks and with the per-token correction, on random
+    shapes: the kept mask against the oracle's rule (ties at the cut
+    counted), and the output against the oracle fed the kernel's kept sets
+    (external-mask mode, so that a tie decided the other way cannot move it)."""
+    from test_gpu_mask import _rule_near
+
+    B, H, d, N, rule, param, n_forced, correction = _case_rules(seed)
+    wl = Workload(f"fr{seed}", B, H, d, (1, 1, N))
+    q, k, v = make_qkv(wl, seed=100 + seed)
+    kw = {"topk": param} if rule == "topk" else ({"topp": param} if rule == "topp" else {})
+    beta = param if rule == "threshold" else 0.0
+    out, lse, dens, mask, _ = forward_with_routing(*(x.cuda() for x in (q, k, v)), beta, rule=rule,
+                                                   n_forced=n_forced, correction=correction, **kw)
+    flips = 0
+    for b in range(B):
+        for h in range(H):
+            r = orc.route_rule(q[b, h].double().numpy(), k[b, h].double().numpy(), rule, param, n_forced)
+            near = _rule_near(r, rule, param, N)
+            if n_forced:
+                assert mask[b, h][:, :min(n_forced, mask.shape[-1])].all()
+                near[:, :n_forced] = False
+            diff = mask[b, h] != r["mask"]
+            assert not (diff & ~near).any(), (seed, b, h, np.argwhere(diff & ~near)[:5])
+            flips += int(diff.sum())
+    assert (dens.cpu().numpy() == mask.sum(-1)).all()
+    out_o, lse_o, _ = orc.forward(q, k, v, beta, masks=mask, correction=correction)
+    og = out.float().cpu().numpy().astype(np.float64)
+    err = og - out_o
+    rel = np.linalg.norm(err) / max(np.linalg.norm(out_o), 1e-30)
+    dl = np.abs(lse.cpu().numpy() - lse_o).max()
+    print(f"B={B} H={H} d={d} N={N} {rule}({param:.3f}) forced={n_forced} {correction}: rel-L2 {rel:.2e} "
+          f"max {np.abs(err).max():.2e} lse {dl:.2e} flipped {flips}")
+    assert rel <= 1e-2 and np.abs(err).max() <= 2e-2 and dl <= 1e-3
