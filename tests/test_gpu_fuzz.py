@@ -112,3 +112,49 @@ def test_random_shapes_other_rules_and_token_correction(seed):
     print(f"B={B} H={H} d={d} N={N} {rule}({param:.3f}) forced={n_forced} {correction}: rel-L2 {rel:.2e} "
           f"max {np.abs(err).max():.2e} lse {dl:.2e} flipped {flips}")
     assert rel <= 1e-2 and np.abs(err).max() <= 2e-2 and dl <= 1e-3
+
+
+@pytest.mark.parametrize("seed", list(range(6)))
+def test_random_strided_layouts(seed):
+    """Random shapes in a strided layout (the [B, N, H, d] order seen through a
+    permute, or rows padded by 8 to 40 elements): pooled statistics and
+    forward outputs equal the contiguous layout's bit for bit, and match the
+    oracle."""
+    import block_sparse_attention_cov_b200 as sa
+
+    rng = np.random.default_rng(3000 + seed)
+    B, H = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+    d = int(rng.choice([64, 128]))
+    N = int(rng.integers(2, 3000))
+    beta = float(rng.normal(0.5, 0.5))
+    pad = int(rng.choice([8, 16, 24, 40]))
+    wl = Workload(f"fs{seed}", B, H, d, (1, 1, N))
+    q, k, v = (x.cuda() for x in make_qkv(wl, seed=200 + seed))
+
+    def view(x):
+        if seed % 2 == 0:
+            return x.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        base = torch.zeros((B, H, N, d + pad), dtype=x.dtype, device=x.device)
+        base[..., :d] = x
+        return base[..., :d]
+
+    st_c = sa.pool(q, k, v)
+    ref = sa.forward(q, k, v, st_c, beta)
+    qs, ks, vs = view(q), view(k), view(v)
+    st_s = sa.pool(qs, ks, vs)
+    out = view(torch.zeros_like(q))
+    got = sa.forward(qs, ks, vs, st_s, beta, out=out)
+    torch.cuda.synchronize()
+    for name in ("qbar", "kbar", "vbar", "kmean", "kcov", "kbar16", "vbar16"):
+        assert torch.equal(st_s.view(name), st_c.view(name)), name  # the alignment gaps are never written
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
+    out_o, lse_o, dens_o = orc.forward(q.cpu(), k.cpu(), v.cpu(), beta)
+    r = orc.route_all(q.cpu(), k.cpu(), beta)
+    ties = (np.abs(r["shat"] - r["tau"][..., None]) <= TIE).sum(-1)
+    diff = np.abs(got[2].cpu().numpy().astype(np.int64) - dens_o)
+    assert (diff[ties == 0] == 0).all() and (diff <= ties).all()
+    err = got[0].float().cpu().numpy().astype(np.float64) - out_o
+    rel = np.linalg.norm(err) / np.linalg.norm(out_o)
+    print(f"B={B} H={H} d={d} N={N} {'bnhd' if seed % 2 == 0 else f'pad {pad}'}: rel-L2 {rel:.2e}")
+    assert rel <= 1e-2 and np.abs(err).max() <= 2e-2
+    assert np.abs(got[1].cpu().numpy() - lse_o).max() <= 1e-3

@@ -45,7 +45,9 @@ def test_strided_layouts_equal_contiguous_bitwise(d, rule):
         assert not qs.is_contiguous()
         st_s = sa.pool(qs, ks, vs)
         torch.cuda.synchronize()
-        assert torch.equal(st_s.buffer, st_c.buffer)  # pooled statistics: same bits
+        for name in ("qbar", "kbar", "vbar", "kmean", "kcov", "kbar16", "vbar16"):
+            # pooled statistics: same bits (the alignment gaps between the arrays are never written)
+            assert torch.equal(st_s.view(name), st_c.view(name)), name
         out = view(torch.zeros_like(q))
         got = sa.forward(qs, ks, vs, st_s, 0.6, out=out, **kw)
         torch.cuda.synchronize()
