@@ -407,9 +407,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 13 || warp == 15) {
     // ======================= MMA issuers: warp 13 = QK, warp 15 = PV =======================
     // QK(t) goes into S slot t % 3 as soon as its K tile has landed and the
-    // PV that last read P from that slot (tile t - 3) has completed: MMAs into
-    // different accumulators are not ordered with each other, so the slot is
-    // reused only after pv_done (waited once per tile, in order). The S ring
+    // PV that last read P from that slot (tile t - 3) has completed: QK and PV
+    // come from different issuer threads, whose MMAs are not ordered with each
+    // other, so the slot is reused only after pv_done (waited once per tile, in
+    // order). The S ring
     // therefore runs up to two tiles ahead of the softmax. PV(t) goes as soon
     // as all eight softmax warps have stored P(t) and its V blocks have landed.
     const bool isQK = warp == 13;
