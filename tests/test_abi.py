@@ -210,3 +210,24 @@ def test_forward_host_argument_errors(L):
     assert L.solattn_forward_host(*args(n=1024)) == _lib.ERR_WORKSPACE
     assert L.solattn_forward_host(p, p, p, 1, 2, 256, 80, f(0.5), p, None, None, 0, scratch, 1 << 30,
                                   None) == _lib.ERR_UNSUPPORTED
+
+
+def test_plain_c_client_compiles_links_and_passes(L, tmp_path):
+    """The boundary is a C ABI: a C program that includes only
+    include/solattn.h and links libsolattn.so compiles with gcc and passes its
+    host-side checks (no GPU needed)."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "c_client"
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c_client.c"), "-L", libdir, "-lsolattn", f"-Wl,-rpath,{libdir}", "-lm",
+           "-o", str(exe)]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    proc = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert proc.returncode == 0, proc.stderr
+    assert "c client ok" in proc.stdout
